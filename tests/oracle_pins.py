@@ -1,0 +1,370 @@
+"""Checks that pin the CPU oracle to facts fixed outside it.
+
+Each ``pin_*`` takes the oracle module and raises AssertionError when the
+oracle disagrees with what the pages, the MX format or plain mathematics
+fix.  ``tests/test_oracle_pins.py`` runs them on the real oracle;
+``tests/test_oracle_mutants.py`` plants typical mistakes in copies of the
+oracle and checks that some pin fails for every one of them.
+
+Nothing here calls the oracle to produce its own expected values: the
+expected side is a closed form, a library routine (numpy.linalg, scipy,
+ml_dtypes, torch dtypes), a brute-force search written here, or a value
+worked out by hand in a comment.
+"""
+from __future__ import annotations
+
+import math
+
+import ml_dtypes
+import numpy as np
+import scipy.linalg
+import torch
+
+import synthetic
+
+RNG_SEED = 1234
+
+
+def _rand_params(nb, seed=RNG_SEED):
+    return synthetic.make_params(nb, seed)
+
+
+# --------------------------------------------------------------------------
+# transform
+# --------------------------------------------------------------------------
+def pin_factor_unit_determinant(o):
+    """Each factor has determinant 1 (unit-determinant LU factors)."""
+    rng = np.random.default_rng(1)
+    for _ in range(200):
+        a, b = rng.normal(0, 2, 2)
+        u = math.exp(rng.normal(0, 1))
+        A = o.lu_factor(a, b, u)
+        assert abs(np.linalg.det(A) - 1.0) < 1e-12, (a, b, u, np.linalg.det(A))
+
+
+def pin_factor_lu_entries(o):
+    """A = L U with L = [[1,0],[a,1]], U = [[u,b],[0,1/u]]: worked by hand,
+    A = [[u, b], [a u, a b + 1/u]]."""
+    a, b, u = 0.75, -1.25, 2.0
+    A = o.lu_factor(a, b, u)
+    want = np.array([[2.0, -1.25], [1.5, 0.75 * -1.25 + 0.5]])
+    assert np.array_equal(A, want), A
+
+
+def pin_block_unit_determinant(o):
+    T = o.expand_params(_rand_params(8))
+    for Tj in T:
+        sign, logdet = np.linalg.slogdet(Tj)
+        assert sign == 1.0 and abs(logdet) < 1e-10, (sign, logdet)
+
+
+def pin_inverse(o):
+    p = _rand_params(6)
+    T = o.expand_params(p)
+    Ti = o.expand_inverse(p)
+    for Tj, Tij in zip(T, Ti):
+        assert np.allclose(Tij @ Tj, np.eye(32), atol=1e-11)
+        ref = np.linalg.inv(Tj)
+        assert np.allclose(Tij, ref, rtol=1e-9, atol=1e-11)
+
+
+def _kron_by_index_bits(p):
+    """T[i][k] = prod_m A_m[bit(i, 4-m)][bit(k, 4-m)], the Kronecker index map
+    written out with the factor built from its definition (not the oracle's)."""
+    p = np.asarray(p, dtype=np.float64).reshape(5, 3)
+    A = []
+    for a, b, u in p:
+        A.append([[u, b], [a * u, a * b + 1.0 / u]])
+    T = np.empty((32, 32))
+    for i in range(32):
+        for k in range(32):
+            v = 1.0
+            for m in range(5):
+                s = 4 - m
+                v *= A[m][(i >> s) & 1][(k >> s) & 1]
+            T[i, k] = v
+    return T
+
+
+def pin_kronecker_index_map(o):
+    p = _rand_params(4, seed=5)
+    T = o.expand_params(p)
+    for j in range(4):
+        ref = _kron_by_index_bits(p[j])
+        assert np.allclose(T[j], ref, rtol=1e-14, atol=0), np.abs(T[j] - ref).max()
+
+
+def pin_param_count(o):
+    """15 parameters per 32-channel block, fewer than half of per-channel
+    scaling's 32 (abstract: 'less than half the parameters')."""
+    assert o.PARAMS_PER_BLOCK == 15
+    assert o.PARAMS_PER_BLOCK * 2 < o.BLOCK
+    assert o.expand_params(np.zeros((1, 15), np.float32) + np.tile([0, 0, 1], 5)).shape == (1, 32, 32)
+
+
+def pin_factor_order(o):
+    """Factor 1 on the most significant index bit: with factor 1 = diag(2, 1/2)
+    and the others identity, T = diag(2 x16, 1/2 x16); factor 5 the same
+    gives diag(2, 1/2, 2, 1/2, ...)."""
+    for m, want in ((0, [2.0] * 16 + [0.5] * 16), (4, [2.0, 0.5] * 16),
+                    (1, ([2.0] * 8 + [0.5] * 8) * 2)):
+        p = np.tile(np.array([0.0, 0.0, 1.0]), 5)
+        p[3 * m + 2] = 2.0
+        T = o.expand_params(p[None])[0]
+        assert np.array_equal(T, np.diag(want)), (m, np.diag(T))
+
+
+def pin_lower_factor_position(o):
+    """Shear a in factor 1 only: T = [[I, 0], [a I, I]] (16x16 blocks); a lower
+    (not upper) triangular L puts a below the diagonal."""
+    p = np.tile(np.array([0.0, 0.0, 1.0]), 5)
+    p[0] = 3.0
+    T = o.expand_params(p[None])[0]
+    want = np.eye(32)
+    want[16:, :16] = 3.0 * np.eye(16)
+    assert np.array_equal(T, want)
+    p = np.tile(np.array([0.0, 0.0, 1.0]), 5)
+    p[3 * 4 + 1] = -2.0     # b of factor 5: upper entry, pairs (2i, 2i+1)
+    T = o.expand_params(p[None])[0]
+    want = np.eye(32)
+    for i in range(0, 32, 2):
+        want[i, i + 1] = -2.0
+    assert np.array_equal(T, want)
+
+
+def pin_rotation_is_hadamard(o):
+    """Five 45-degree rotations R = [[c, -s], [s, c]] (u = c, b = -s, a = s/c = 1)
+    give T = H_32 diag((-1)^popcount(k)) / sqrt(32), H_32 Sylvester's Hadamard
+    matrix (scipy), because R = H_2 diag(1, -1) / sqrt(2)."""
+    c = 1.0 / math.sqrt(2.0)
+    p = np.tile(np.array([1.0, -c, c]), 5)
+    T = o.expand_params(p[None])[0]
+    H = scipy.linalg.hadamard(32).astype(np.float64)
+    D = np.diag([(-1.0) ** bin(k).count("1") for k in range(32)])
+    assert np.allclose(T, H @ D / math.sqrt(32), atol=1e-14)
+    x = np.random.default_rng(3).normal(size=(5, 64))
+    y = o.transform(x, np.stack([p, p]))
+    # FWHT of the sign-flipped input, by the textbook in-place butterfly
+    for r in range(5):
+        for j in range(2):
+            v = x[r, 32 * j:32 * j + 32] * np.diag(D)
+            h = 1
+            v = v.copy()
+            while h < 32:
+                for i in range(0, 32, 2 * h):
+                    for k in range(i, i + h):
+                        v[k], v[k + h] = v[k] + v[k + h], v[k] - v[k + h]
+                h *= 2
+            assert np.allclose(y[r, 32 * j:32 * j + 32], v / math.sqrt(32), atol=1e-12)
+
+
+def pin_identity_params(o):
+    nb = 3
+    p = synthetic.identity_params(nb)
+    assert np.array_equal(o.expand_params(p), np.stack([np.eye(32)] * nb))
+    x = np.random.default_rng(4).normal(size=(7, 32 * nb)) * 3
+    assert np.array_equal(o.transform(x, p), x)
+
+
+def pin_transform_column_convention(o):
+    """y = T x per token (x a column vector): with only b of factor 1 set,
+    y[i] = x[i] + b x[i + 16] for i < 16 and y[i] = x[i] above."""
+    p = np.tile(np.array([0.0, 0.0, 1.0]), 5)
+    p[1] = 0.5
+    x = np.arange(32, dtype=np.float64)[None]
+    y = o.transform(x, p[None])[0]
+    want = x[0].copy()
+    want[:16] += 0.5 * x[0, 16:]
+    assert np.array_equal(y, want), y
+
+
+# --------------------------------------------------------------------------
+# MXFP4
+# --------------------------------------------------------------------------
+def _ml_code(v):
+    q = np.asarray(v, dtype=np.float32).astype(ml_dtypes.float4_e2m1fn)
+    return q.view(np.uint8) & 0xF
+
+
+def pin_e2m1_grid(o):
+    codes = np.arange(16, dtype=np.uint8)
+    ml = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(o.e2m1_decode(codes), ml)
+    assert set(np.abs(o.e2m1_decode(codes))) == {0, 0.5, 1, 1.5, 2, 3, 4, 6}
+
+
+def _brute_e2m1(r):
+    """Nearest of the 16 codes; ties to the code with mantissa bit 0; beyond 6
+    saturate; the sign bit copies r's sign (so -0.1 gives 0x8)."""
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    m = abs(r)
+    best, bestd = None, None
+    for c in range(8):
+        dd = abs(mags[c] - m)
+        if best is None or dd < bestd - 1e-300 or (dd == bestd and (c & 1) == 0):
+            best, bestd = c, dd
+    sign = 1 if math.copysign(1.0, r) < 0 else 0
+    return sign << 3 | best
+
+
+def _edge_values():
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    vals = []
+    for m in mids + grid + [6.5, 7.0, 7.5, 7.999, 8.0, 100.0, 1e-30]:
+        for eps in (0.0, 1e-6, -1e-6, 2.0 ** -20, -(2.0 ** -20)):
+            v = m + eps
+            if v >= 0:
+                vals += [v, -v]
+    return np.array(vals + [-0.0, 0.0])
+
+
+def pin_e2m1_rounding(o):
+    vals = np.concatenate([_edge_values(),
+                           np.random.default_rng(6).uniform(-9, 9, 4000)]).astype(np.float32)
+    got = o.e2m1_code(vals.astype(np.float64))
+    assert np.array_equal(got, _ml_code(vals)), vals[got != _ml_code(vals)]
+    brute = np.array([_brute_e2m1(float(v)) for v in vals], dtype=np.uint8)
+    assert np.array_equal(got, brute), vals[got != brute]
+
+
+def pin_e8m0(o):
+    bytes_ = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(bytes_).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    got = o.e8m0_decode(bytes_)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+
+
+def pin_shared_exponent(o):
+    """floor(log2(amax)) - 2, clamped to [-127, 127]; worked by hand."""
+    cases = {1.0: -2, 6.0: 0, 7.99: 0, 8.0: 1, 4.0: 0, 3.999: -1, 0.5: -3,
+             2.0 ** 100: 98, 2.0 ** 200: 127, 0.0: -127, 2.0 ** -126: -127,
+             2.0 ** -124: -126, 2.0 ** -125: -127, 5e-324: -127}
+    for amax, e in cases.items():
+        got = int(o.shared_exponent(np.array([amax]))[0])
+        assert got == e, (amax, got, e)
+
+
+def pin_hand_block(o):
+    """One block worked by hand.  Values (then padded with zeros):
+      x = [6, -7.5, 0.3, -0.2, 1.25, 2.5, 3.5, 5, -0.75, 0.74, ...]
+    amax = 7.5 -> floor(log2 7.5) = 2 -> e = 0, scale byte 127, r = x.
+      6 -> 6 (0x7); -7.5 -> saturates -6 (0xF); 0.3 -> 0.5 (0x1);
+      -0.2 -> -0 (0x8); 1.25 tie -> 1.0 (0x2); 2.5 tie -> 2 (0x4);
+      3.5 tie -> 4 (0x6); 5 tie -> 4 (0x6); -0.75 tie -> -1.0 (0xA);
+      0.74 -> 0.5 (0x1); zeros -> 0x0.
+    Bytes pack (even element low nibble): 0xF7, 0x81, 0x42, 0x66, 0x1A, 0, ..."""
+    x = np.zeros((1, 32))
+    x[0, :10] = [6, -7.5, 0.3, -0.2, 1.25, 2.5, 3.5, 5, -0.75, 0.74]
+    codes, scales = o.quantize_mxfp4(x)
+    assert scales.tolist() == [[127]]
+    assert codes[0, :5].tolist() == [0xF7, 0x81, 0x42, 0x66, 0x1A]
+    assert not codes[0, 5:].any()
+    # scaled copy: x * 2**-10 only moves the scale byte by -10
+    codes2, scales2 = o.quantize_mxfp4(x * 2.0 ** -10)
+    assert scales2.tolist() == [[117]] and np.array_equal(codes2, codes)
+    # all-zero block: byte 0 (2**-127), codes 0
+    codes3, scales3 = o.quantize_mxfp4(np.zeros((1, 32)))
+    assert scales3.tolist() == [[0]] and not codes3.any()
+    # NaN anywhere: byte 0xFF
+    xn = x.copy()
+    xn[0, 31] = np.nan
+    assert o.quantize_mxfp4(xn)[1].tolist() == [[255]]
+    xi = x.copy()
+    xi[0, 3] = -np.inf
+    assert o.quantize_mxfp4(xi)[1].tolist() == [[255]]
+
+
+def pin_brute_pipeline(o):
+    """A few blocks of the tiny workload, every step by plain loops in fp64:
+    T from the index-bit product, y from explicit sums, amax, frexp exponent,
+    brute-force code search, nibble packing."""
+    w = synthetic.CONFIGS["tiny"][0]
+    raw = synthetic.make_activations(w, rows=[0, 77, 255])
+    x = raw.astype(np.float64)
+    p = synthetic.make_params(w.nb, w.seed)
+    codes, scales = o.kq_quantize(x, p)
+    for j in (0, 7, 35):
+        T = _kron_by_index_bits(p[j])
+        for r in range(3):
+            xb = x[r, 32 * j:32 * j + 32]
+            y = [math.fsum(T[i, k] * xb[k] for k in range(32)) for i in range(32)]
+            amax = max(abs(v) for v in y)
+            e = max(-127, min(127, math.frexp(amax)[1] - 1 - 2)) if amax > 0 else -127
+            assert scales[r, j] == e + 127
+            nib = [_brute_e2m1(v / 2.0 ** e) for v in y]
+            packed = [nib[2 * i] | nib[2 * i + 1] << 4 for i in range(16)]
+            assert codes[r, 16 * j:16 * j + 16].tolist() == packed, (r, j)
+
+
+def pin_roundtrip_bound(o):
+    """dequant(quant(y)) differs from y by at most half a grid step at r
+    (0.25, 0.5, 1 in binades [0,2), [2,4), [4,6]) or by |r| - 6 when
+    saturated, times 2**e; undoing T then bounds the error in x."""
+    w = synthetic.CONFIGS["tiny"][0]
+    x = synthetic.make_activations(w, rows=np.arange(64)).astype(np.float64)
+    p = synthetic.make_params(w.nb, w.seed)
+    y = o.transform(x, p)
+    codes, scales = o.quantize_mxfp4(y)
+    deq = o.dequant(codes, scales)
+    M, d = y.shape
+    e = (scales.astype(np.int64) - 127).repeat(32, axis=1)
+    r = np.abs(y) / 2.0 ** e
+    half = np.where(r < 2, 0.25, np.where(r < 4, 0.5, 1.0))
+    bound = np.where(r > 6, r - 6, half) * 2.0 ** e
+    assert np.all(np.abs(deq - y) <= bound * (1 + 1e-12))
+    Tinv = o.expand_inverse(p)
+    xr = o.apply_blockdiag(deq, Tinv)
+    xb = o.apply_blockdiag(bound, np.abs(Tinv))
+    assert np.all(np.abs(xr - x) <= xb * (1 + 1e-9) + 1e-12)
+
+
+def pin_fold_invariance(o):
+    """W' (T x) = W x for W' = fold(W)."""
+    nb = 4
+    p = _rand_params(nb, seed=11)
+    W = synthetic.make_weights(24, 32 * nb, 3).astype(np.float64)
+    x = np.random.default_rng(12).normal(size=(32 * nb, 5))
+    Wf = o.fold_weights(W, p)
+    Tx = o.transform(x.T, p).T
+    lhs = Wf @ Tx
+    rhs = W @ x
+    assert np.allclose(lhs, rhs, rtol=1e-10, atol=1e-10 * np.abs(rhs).max())
+
+
+def pin_smoothquant_is_diagonal_case(o):
+    """a = b = 0 makes T diagonal; SmoothQuant with 1/s = diag(T) then gives
+    the same codes and scales."""
+    nb = 3
+    p = _rand_params(nb, seed=21).reshape(nb, 5, 3).copy()
+    p[:, :, 0] = 0
+    p[:, :, 1] = 0
+    p = p.reshape(nb, 15)
+    T = o.expand_params(p)
+    diag = np.concatenate([np.diag(t) for t in T])
+    x = synthetic.f32_from_bf16_bits(
+        synthetic.bf16_bits_from_f32(np.random.default_rng(2).normal(size=(9, 96)).astype(np.float32))
+    ).astype(np.float64)
+    c1, s1 = o.kq_quantize(x, p)
+    c2, s2 = o.sq_quantize(x, diag)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def pin_undecided_flags(o):
+    y = np.zeros((1, 32))
+    y[0, 0] = 4.0 * 1.25          # amax 5 -> e = 0; r = 5 is a midpoint
+    y[0, 1] = 1.3                 # far from any midpoint
+    y[0, 2] = 0.25 * (1 + 5e-5)   # within 1e-4 relative of 0.25
+    tol = np.full((1, 32), 1e-9)
+    elem, blk = o.undecided(y, tol)
+    assert elem[0, 0] and not elem[0, 1] and elem[0, 2]
+    assert not blk[0, 0]
+    y2 = y.copy()
+    y2[0, 0] = 4.0 * (1 + 1e-6)   # amax next to a power of two
+    elem2, blk2 = o.undecided(y2, tol)
+    assert blk2[0, 0] and elem2.all()
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
