@@ -1,0 +1,536 @@
+#!/usr/bin/env python
+"""Throughput of the KroQuant online activation quantizer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kroquant|reference]
+
+A step quantizes one batch of the FLUX.1-schnell-shaped workload: the
+activations entering the attention projections (M = 4608 tokens x d = 3072)
+and the MLP output projection (4608 x 12288), bf16 in, MXFP4 (E2M1 codes +
+E8M0 scales) out, one ``kq_quantize`` launch each.  Inputs are synthetic
+(seeded, with the workload's outlier channels and per-token mean shift) and
+resident in HBM before the timed region; consecutive steps cycle through a
+ring of distinct input/output buffers whose total exceeds 4x the L2 size,
+so no step reads what the previous one left in L2.
+
+The metric is GB/s of algorithmic traffic (2 B read + 0.5 B codes + 1/32 B
+scale per element, plus 60 B of parameters per 32-channel block column and
+launch), timed with CUDA events on the launching stream, max over ranks.
+Under torchrun each rank (one per GPU) quantizes its own tokens: the path
+has no exchange step, so there is no collective beyond the barrier and the
+max-reduce of the timings (weak scaling).
+
+``--impl reference`` times the CPU oracle (fp64 NumPy, single thread) on a
+bounded sample of the same workload instead; rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synthetic  # noqa: E402
+
+METRIC = "kq_quantize GB/s (bf16 in→MXFP4 out) and % of B200 HBM peak, vs SmoothQuant"
+UNIT = "GB/s"
+WORKLOAD = "flux"
+BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
+PARAM_BYTES_PER_BLOCK_COL = 15 * 4
+FALLBACK_HBM_GBS = 6650.0
+RING_FACTOR_L2 = 4.0
+PAGES_CONTEXT = ("the pages report the KroQuant quantizer kernel up to 14% faster than "
+                 "the SmoothQuant kernel on AMD MI350 (relative only; shapes not given)")
+
+
+# ---------------------------------------------------------------------------
+# workload and rank plan
+# ---------------------------------------------------------------------------
+def step_workloads(rank: int = 0) -> list[synthetic.Workload]:
+    """The shapes one step quantizes on `rank`.  Each rank owns its own tokens
+    (a different seed), same shapes: weak scaling."""
+    import dataclasses
+    out = []
+    for w in synthetic.CONFIGS[WORKLOAD]:
+        out.append(dataclasses.replace(w, seed=w.seed + 1000 * rank) if rank else w)
+    return out
+
+
+def algorithmic_bytes(M: int, d: int) -> float:
+    return M * d * BYTES_PER_ELEM + (d // 32) * PARAM_BYTES_PER_BLOCK_COL
+
+
+def step_bytes(ws) -> float:
+    return sum(algorithmic_bytes(w.M, w.d) for w in ws)
+
+
+def ring_depth(ws, l2_bytes: int) -> int:
+    per_step = sum(w.M * w.d * (2 + 0.5 + 1 / 32) for w in ws)
+    return max(2, int(math.ceil(RING_FACTOR_L2 * l2_bytes / per_step)))
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML)
+# ---------------------------------------------------------------------------
+REASON_BITS = {
+    "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+    "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+    "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+}
+
+
+class ClockSampler:
+    """Polls the SM clock and the clock-event reasons of one GPU in a thread."""
+
+    def __init__(self, index: int, period_s: float = 0.0005):
+        self.samples = []          # (t, sm_mhz, reasons)
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report clocks as unavailable
+            self._nv = None
+            self.error = f"{type(e).__name__}: {e}"
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join(timeout=2)
+
+    def summary(self, t0: float, t1: float) -> dict:
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.error}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(win) < 3:
+            win = self.samples
+            window = "warm-up and timed region (timed region shorter than the sampling period)"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "note": "no samples"}
+        mask = 0
+        for _, _, r in win:
+            mask |= int(r)
+        reasons = [k for k, b in REASON_BITS.items() if mask & b and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(win), "window": window}
+
+
+# ---------------------------------------------------------------------------
+# roofline inputs
+# ---------------------------------------------------------------------------
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs: STREAM-style copy on this pool's B200s)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def ncu_traffic():
+    """DRAM bytes per launch of the d=12288 kq_quantize launch from the
+    committed ncu summary, if it was taken on the current sources."""
+    path = os.path.join(ROOT, "profiles", "kq_quantize_flux.md")
+    try:
+        from w4a4_dit_post_b200 import build
+        cur = build.source_hash()
+        vals = {}
+        with open(path) as f:
+            for line in f:
+                if line.startswith("<!-- ") and "=" in line:
+                    k, v = line[5:].split("-->")[0].strip().split("=", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("source_hash") == cur and "traffic_bytes_per_launch" in vals:
+            return float(vals["traffic_bytes_per_launch"]), "ncu (current sources)"
+        return None, "ncu summary predates the current kernel sources"
+    except Exception as e:
+        return None, f"no ncu summary ({type(e).__name__})"
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def run_kroquant(args) -> int:
+    import torch
+
+    import w4a4_dit_post_b200 as kq
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    props = torch.cuda.get_device_properties(device)
+    l2 = int(getattr(props, "L2_cache_size", 0) or 126 * 2 ** 20)
+
+    ws = step_workloads(rank)
+    R = ring_depth(ws, l2)
+    stream = torch.cuda.current_stream(device)
+
+    # inputs: the seeded workload, then R-1 row rotations of it (distinct buffers)
+    rings = []
+    host_pinned = []
+    for w in ws:
+        raw = synthetic.make_activations(w)
+        host = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16)
+        pinned = torch.empty_like(host).pin_memory()
+        pinned.copy_(host)
+        host_pinned.append(pinned)
+        x0 = pinned.to(device)
+        p = torch.from_numpy(synthetic.make_params(w.nb, w.seed)).to(device)
+        inv_s = torch.from_numpy(synthetic.smoothquant_inv_scales(
+            synthetic.f32_from_bf16_bits(raw[:: max(1, w.M // 1024)]))).to(device)
+        slots = []
+        for r in range(R):
+            x = x0 if r == 0 else torch.roll(x0, shifts=r * 997, dims=0).contiguous()
+            codes = torch.empty((w.M, w.d // 2), dtype=torch.uint8, device=device)
+            scales = torch.empty((w.M, w.d // 32), dtype=torch.uint8, device=device)
+            slots.append((x, codes, scales))
+        rings.append((w, p, inv_s, slots))
+        del raw, host
+    torch.cuda.synchronize(device)
+    kq.kq_device_status(device, clear=True)
+
+    dominant = max(range(len(ws)), key=lambda i: ws[i].M * ws[i].d)
+
+    def one_step(k, fn, ev=None):
+        for i, (w, p, inv_s, slots) in enumerate(rings):
+            x, codes, scales = slots[k % R]
+            if ev is not None:
+                ev[i][0][k].record(stream)
+            if fn == "kq":
+                kq.kq_quantize(x, p, codes, scales)
+            else:
+                kq.sq_quantize(x, inv_s, codes, scales)
+            if ev is not None:
+                ev[i][1][k].record(stream)
+
+    def timed(fn, K, W, per_launch=False):
+        for k in range(W):
+            one_step(k, fn)
+        ev = None
+        if per_launch:
+            ev = [([torch.cuda.Event(enable_timing=True) for _ in range(K)],
+                   [torch.cuda.Event(enable_timing=True) for _ in range(K)]) for _ in rings]
+        barrier(world, device)
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        e0.record(stream)
+        for k in range(K):
+            one_step(W + k, fn, ev)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        t1 = time.perf_counter()
+        barrier(world, device)
+        ms = e0.elapsed_time(e1)
+        launch_ms = None
+        if per_launch:
+            launch_ms = [sum(a.elapsed_time(b) for a, b in zip(ev[i][0], ev[i][1])) / K
+                         for i in range(len(rings))]
+        return ms, launch_ms, t0, t1
+
+    K, W = args.steps, args.warmup
+    sampler = ClockSampler(device.index if device.index is not None else 0).start()
+    ms_kq, launch_kq, t0, t1 = timed("kq", K, W, per_launch=True)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    ms_sq, launch_sq, _, _ = timed("sq", K, W, per_launch=True)
+
+    # end to end through the public API: pinned host input -> device -> quantize -> host
+    host_out = [(torch.empty((w.M, w.d // 2), dtype=torch.uint8).pin_memory(),
+                 torch.empty((w.M, w.d // 32), dtype=torch.uint8).pin_memory()) for w in ws]
+
+    def e2e_step(k):
+        for i, (w, p, _, slots) in enumerate(rings):
+            x, codes, scales = slots[k % R]
+            x.copy_(host_pinned[i], non_blocking=True)
+            kq.kq_quantize(x, p, codes, scales)
+            host_out[i][0].copy_(codes, non_blocking=True)
+            host_out[i][1].copy_(scales, non_blocking=True)
+
+    for k in range(W):
+        e2e_step(k)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for k in range(K):
+        e2e_step(W + k)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    ms_e2e = a.elapsed_time(b)
+
+    status = kq.kq_device_status(device)
+    sbytes = step_bytes(ws)
+    total_bytes = sum_over_ranks(sbytes * K, world, device)
+    ms_kq_max = max_over_ranks(ms_kq, world, device)
+    ms_sq_max = max_over_ranks(ms_sq, world, device)
+    ms_e2e_max = max_over_ranks(ms_e2e, world, device)
+
+    if rank == 0:
+        value = total_bytes / (ms_kq_max * 1e-3) / 1e9
+        sq_value = total_bytes / (ms_sq_max * 1e-3) / 1e9
+        e2e_value = total_bytes / (ms_e2e_max * 1e-3) / 1e9
+        peak, peak_src = hbm_peak()
+        wd = ws[dominant]
+        dom_bytes = algorithmic_bytes(wd.M, wd.d)
+        achieved = dom_bytes / (launch_kq[dominant] * 1e-3) / 1e9
+        traffic, traffic_src = ncu_traffic()
+        per_shape = {}
+        for i, w in enumerate(ws):
+            bts = algorithmic_bytes(w.M, w.d)
+            per_shape[f"{w.M}x{w.d}"] = {
+                "kq_us": round(launch_kq[i] * 1e3, 2),
+                "kq_gbs": round(bts / (launch_kq[i] * 1e-3) / 1e9, 1),
+                "kq_frac_of_peak": round(bts / (launch_kq[i] * 1e-3) / 1e9 / peak, 4),
+                "sq_us": round(launch_sq[i] * 1e3, 2),
+                "sq_gbs": round(bts / (launch_sq[i] * 1e-3) / 1e9, 1),
+            }
+        line = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": K,
+            "warmup": W,
+            "ms_per_step": round(ms_kq_max / K, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded FLUX.1-schnell-shaped activations: N(0,1), 1% outlier "
+                    "channels x100, per-token mean N(0,4); random LU parameters)",
+            "config": {
+                "workload": "FLUX.1-schnell-shaped linear-layer inputs: M=4608 tokens x d in "
+                            "{3072, 12288}, bf16 in -> MXFP4 (E2M1 codes + E8M0 scales) out; "
+                            "one kq_quantize launch per shape per step",
+                "M_per_rank": ws[0].M,
+                "d": [w.d for w in ws],
+                "l2": f"inputs larger than L2: ring of {R} distinct input/output sets "
+                      f"({R * step_bytes(ws) / 1e6:.0f} MB > {RING_FACTOR_L2:.0f} x L2 "
+                      f"{l2 / 2 ** 20:.0f} MiB)",
+                "parallelism": f"replicas x{world} (token rows per rank, no collective)",
+            },
+            "gpu_launches": K * len(ws),
+            "roofline": {
+                "bound": "hbm",
+                "kernel": f"kq_quantize {wd.M}x{wd.d}",
+                "achieved": round(achieved, 1),
+                "peak": peak,
+                "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": traffic,
+                "algorithmic_bytes_per_launch": dom_bytes,
+                "peak_source": peak_src,
+                "traffic_source": traffic_src,
+            },
+            "smoothquant": {
+                "value": round(sq_value, 1),
+                "unit": UNIT,
+                "kq_over_sq_time": round(ms_kq_max / ms_sq_max, 4),
+                "context": PAGES_CONTEXT,
+            },
+            "per_shape": per_shape,
+            "e2e": {
+                "value": round(e2e_value, 2),
+                "unit": UNIT,
+                "h2d_bytes_per_step": int(sum(w.M * w.d * 2 for w in ws)),
+                "d2h_bytes_per_step": int(sum(w.M * w.d // 2 + w.M * w.d // 32 for w in ws)),
+                "path": "pinned host bf16 -> device copy -> kq_quantize (Python binding over the "
+                        "C ABI) -> device-to-host copy of codes and scales, same stream",
+            },
+            "clocks": clocks,
+            "device_status": status,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def _oracle_sample(ws, rows_per_shape: int):
+    """Time the oracle on the first rows of each shape; returns (seconds, bytes)."""
+    import oracle.kq_oracle as o
+    secs = 0.0
+    nbytes = 0.0
+    for w in ws:
+        rows = np.arange(min(rows_per_shape, w.M))
+        x = synthetic.f32_from_bf16_bits(synthetic.make_activations(w, rows)).astype(np.float64)
+        p = synthetic.make_params(w.nb, w.seed)
+        t = time.perf_counter()
+        o.kq_quantize(x, p)
+        secs += time.perf_counter() - t
+        nbytes += rows.size * w.d * BYTES_PER_ELEM + (w.d // 32) * PARAM_BYTES_PER_BLOCK_COL
+    return secs, nbytes
+
+
+def _single_thread():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=1)
+    except Exception:
+        import contextlib
+        return contextlib.nullcontext()
+
+
+def cpu_baseline(seconds: float = 15.0) -> dict:
+    ws = step_workloads(0)
+    with _single_thread():
+        s, b = _oracle_sample(ws, 16)                      # calibrate
+        rows = int(max(16, min(4608, 16 * seconds / max(s, 1e-3))))
+        s, b = _oracle_sample(ws, rows)
+    return {"value": round(b / s / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of 4608 tokens of each FLUX shape (3072, 12288), fp64 NumPy "
+                      f"oracle, one thread, {s:.1f} s"}
+
+
+def run_reference(args) -> int:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    ws = step_workloads(0)
+    with _single_thread():
+        s, _ = _oracle_sample(ws, 8)
+        budget = 150.0 / max(1, args.steps + args.warmup)   # whole run within a few minutes
+        rows = int(max(8, min(4608, 8 * budget / max(s, 1e-3))))
+        for _ in range(args.warmup):
+            _oracle_sample(ws, rows)
+        tot_s, tot_b = 0.0, 0.0
+        for _ in range(args.steps):
+            s, b = _oracle_sample(ws, rows)
+            tot_s += s
+            tot_b += b
+    value = tot_b / tot_s / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot_s / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded FLUX.1-schnell-shaped activations)",
+        "config": {"workload": "FLUX.1-schnell-shaped linear-layer inputs: M=4608 tokens x d in "
+                               "{3072, 12288}, bf16 in -> MXFP4 out; each step a bounded sample "
+                               f"of {rows} tokens per shape",
+                   "M_per_rank": 4608, "d": [w.d for w in ws]},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"first {rows} tokens of each FLUX shape per step"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description="KroQuant quantizer throughput")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["kroquant", "reference"], default="kroquant")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
+    _, world, _ = dist_env()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_kroquant(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,88 @@
+"""Comparison of the CUDA quantizer's output with the CPU oracle.
+
+The tolerance comes from the arithmetic: the kernel evaluates the transform in
+fp32, so each transformed value may differ from the exact (fp64) one by at
+most TOL_REL times the sum of the magnitudes of the terms that make it up,
+sum_k ((x)_m |L_m||U_m|)[i, k] |x_k| (``oracle.error_scale``).  MXFP4 codes
+and scale bytes must then be bit-identical, except for the decisions the
+oracle flags as open within that tolerance or within 1e-4 (relative) of a
+rounding or scale boundary (``oracle.undecided``).  NaN blocks must carry the
+NaN scale byte on both sides; their codes are unspecified.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+import oracle.kq_oracle as o
+
+TOL_REL = 1e-5        # transformed values: fp32 accumulation
+BOUNDARY_REL = 1e-4   # codes / scales: exemption window around a boundary
+
+
+@dataclasses.dataclass
+class Report:
+    n_elems: int
+    n_blocks: int
+    y_violations: int = 0           # |y_gpu - y_ref| > tol (transform check only)
+    scale_mismatch: int = 0         # decided blocks whose byte differs
+    code_mismatch: int = 0          # decided elements whose nibble differs
+    exempt_blocks: int = 0
+    exempt_elems: int = 0
+    differing_exempt: int = 0       # exempt elements that did differ (informational)
+
+    @property
+    def ok(self) -> bool:
+        return self.y_violations == 0 and self.scale_mismatch == 0 and self.code_mismatch == 0
+
+
+def reference(x: np.ndarray, params=None, inv_s=None):
+    """(y_ref, tol) for KroQuant (params) or SmoothQuant (inv_s)."""
+    x = np.asarray(x, dtype=np.float64)
+    if params is not None:
+        y = o.transform(x, params)
+        tol = TOL_REL * o.error_scale(x, params)
+    else:
+        y = o.sq_transform(x, inv_s)
+        tol = TOL_REL * np.abs(y)
+    return y, tol
+
+
+def compare_codes(codes, scales, y_ref, tol, exact: bool = False) -> Report:
+    """Compare GPU (codes, scales) against the oracle's encoding of y_ref.
+    exact=True: every decision must match (inputs whose transform is exact)."""
+    codes = np.asarray(codes)
+    scales = np.asarray(scales)
+    c_ref, s_ref = o.quantize_mxfp4(y_ref)
+    M, d = y_ref.shape
+    rep = Report(n_elems=M * d, n_blocks=M * d // 32)
+    nan_blk = s_ref == o.E8M0_NAN
+    rep.scale_mismatch += int(np.sum(nan_blk & (scales != o.E8M0_NAN)))
+    if exact:
+        e_flags = np.zeros((M, d), dtype=bool)
+        b_flags = np.zeros((M, d // 32), dtype=bool)
+        # only the sign of an exact zero is open
+        e_flags |= (y_ref == 0)
+    else:
+        finite = np.where(np.isfinite(y_ref), y_ref, 0.0)
+        e_flags, b_flags = o.undecided(finite, np.where(np.isfinite(tol), tol, 0.0))
+    rep.exempt_blocks = int(np.sum(b_flags & ~nan_blk))
+    decided_blk = ~b_flags & ~nan_blk
+    rep.scale_mismatch += int(np.sum(decided_blk & (scales != s_ref)))
+    n_gpu = o.unpack_nibbles(codes)
+    n_ref = o.unpack_nibbles(c_ref)
+    same_scale = np.repeat((scales == s_ref) & ~nan_blk, 32, axis=1)
+    elem_decided = ~e_flags & same_scale
+    rep.exempt_elems = int(np.sum(e_flags & np.repeat(~nan_blk, 32, axis=1)))
+    rep.code_mismatch = int(np.sum(elem_decided & (n_gpu != n_ref)))
+    rep.differing_exempt = int(np.sum(~elem_decided & same_scale & (n_gpu != n_ref)))
+    return rep
+
+
+def compare_transform(y_gpu, y_ref, tol) -> Report:
+    y_gpu = np.asarray(y_gpu, dtype=np.float64)
+    M, d = y_ref.shape
+    rep = Report(n_elems=M * d, n_blocks=M * d // 32)
+    rep.y_violations = int(np.sum(~(np.abs(y_gpu - y_ref) <= tol)))
+    return rep

@@ -1,0 +1,107 @@
+"""The C-ABI library without a GPU: it builds for sm_100a, loads, exports
+every function include/kq.h declares, and rejects bad arguments on the host
+with the documented status before touching the device.  No compute call is
+made here (arguments that pass the checks are only used with M == 0)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a4_dit_post_b200 import build
+    build.build()
+    import w4a4_dit_post_b200 as k
+    return k.abi()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**((?:kq|sq)_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_abi():
+    names = header_functions()
+    for want in ("kq_quantize", "kq_transform", "sq_quantize", "kq_expand_params",
+                 "kq_fold_weights", "kq_dequant", "kq_status_string", "kq_device_status"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    import w4a4_dit_post_b200 as k
+    names = header_functions()
+    assert sorted(k.EXPORTED_FUNCTIONS) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_is_sm100a(lib):
+    from w4a4_dit_post_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.ARCH_FLAGS)
+    assert build.is_current()
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = lib.kq_status_string(code).decode()
+        assert s.startswith("KQ_")
+    assert lib.kq_status_string(99).decode()
+    assert lib.kq_version() == 10000
+
+
+# fake, suitably aligned device addresses: never dereferenced by these calls
+A16 = 0x7F0000000000
+A16b = 0x7F0000100000
+A16c = 0x7F0000200000
+A16d = 0x7F0000300000
+
+
+def test_quantize_argument_checks(lib):
+    q = lib.kq_quantize
+    assert q(None, 0, 4, 64, A16b, A16c, A16d, None) == 1          # NULL x
+    assert q(A16, 0, 4, 64, None, A16c, A16d, None) == 1           # NULL params
+    assert q(A16, 0, 4, 64, A16b, None, A16d, None) == 1           # NULL codes
+    assert q(A16, 0, 4, 64, A16b, A16c, None, None) == 1           # NULL scales
+    assert q(A16, 0, -1, 64, A16b, A16c, A16d, None) == 1          # M < 0
+    assert q(A16, 0, 4, 48, A16b, A16c, A16d, None) == 1           # d % 32
+    assert q(A16, 0, 4, 0, A16b, A16c, A16d, None) == 1            # d == 0
+    assert q(A16, 7, 4, 64, A16b, A16c, A16d, None) == 3           # dtype
+    assert q(A16 + 8, 0, 4, 64, A16b, A16c, A16d, None) == 2       # x alignment
+    assert q(A16, 0, 4, 64, A16b + 2, A16c, A16d, None) == 2       # params alignment
+    assert q(A16, 0, 4, 64, A16b, A16c + 4, A16d, None) == 2       # codes alignment
+    assert q(A16, 0, 4, 32768 + 32, A16b, A16c, A16d, None) == 4   # d limit
+    assert q(A16, 0, 2 ** 40, 1024, A16b, A16c, A16d, None) == 4   # block count
+    assert q(A16, 0, 0, 64, A16b, A16c, A16d + 1, None) == 0       # M == 0: no-op
+    assert b"kq_quantize" in lib.kq_last_error()
+
+
+def test_other_argument_checks(lib):
+    assert lib.kq_transform(A16, 0, 4, 64, A16b, A16c + 4, None) == 2
+    assert lib.kq_transform(A16, 1, 0, 64, A16b, A16c, None) == 0
+    assert lib.sq_quantize(A16, 0, 4, 33, A16b, A16c, A16d, None) == 1
+    assert lib.sq_quantize(A16, 1, 0, 64, A16b, A16c, A16d, None) == 0
+    assert lib.kq_expand_params(None, 64, A16, None) == 1
+    assert lib.kq_expand_params(A16, 40, A16b, None) == 1
+    assert lib.kq_fold_weights(A16, 4, 64, A16b, A16 + 8, None) == 2
+    assert lib.kq_fold_weights(A16, 4, 64, A16b, A16 + 64, None) == 1   # partial overlap
+    assert lib.kq_fold_weights(A16, 0, 64, A16b, A16c, None) == 0
+    assert lib.kq_dequant(A16, A16b, 4, 64, A16c + 4, None) == 2
+    assert lib.kq_dequant(A16, A16b, 0, 64, A16c, None) == 0
+    assert lib.kq_device_status(None, 0) == 1
+
+
+def test_binding_refuses_host_tensors(lib):
+    import torch
+    import w4a4_dit_post_b200 as k
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    p = torch.zeros(2, 15)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        k.kq_quantize(x, p)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        k.kq_dequant(torch.zeros(4, 32, dtype=torch.uint8), torch.zeros(4, 2, dtype=torch.uint8))

@@ -1,0 +1,207 @@
+"""Python binding of the KroQuant C ABI (``include/kq.h``, ``libkroquant.so``).
+
+Argument marshalling only: every function checks that it was handed CUDA
+tensors of the right dtype and shape, allocates missing outputs with torch
+(device memory is PyTorch's job here), and passes raw device pointers and the
+current torch stream to the C function of the same name.  All arithmetic runs
+in the library's sm_100a kernels; there is no CPU path.  If the library has
+not been built, the first call raises ``RuntimeError`` (build it with
+``python -m w4a4_dit_post_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from .build import LIB_PATH
+
+__all__ = [
+    "abi", "kq_quantize", "kq_transform", "sq_quantize", "kq_expand_params",
+    "kq_fold_weights", "kq_dequant", "kq_device_status", "KroQuantError",
+    "KQ_DTYPE_BF16", "KQ_DTYPE_F32", "KQ_MAX_D", "EXPORTED_FUNCTIONS",
+]
+
+KQ_OK = 0
+KQ_DTYPE_BF16 = 0
+KQ_DTYPE_F32 = 1
+KQ_MAX_D = 32768
+
+_c_void_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+# name -> (restype, argtypes), mirroring include/kq.h
+_SIGNATURES = {
+    "kq_quantize": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "kq_transform": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "sq_quantize": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "kq_expand_params": (_int, [_c_void_p, _i64, _c_void_p, _c_void_p]),
+    "kq_fold_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "kq_dequant": (_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
+    "kq_device_status": (_int, [ctypes.POINTER(ctypes.c_uint32), _int]),
+    "kq_status_string": (ctypes.c_char_p, [_int]),
+    "kq_last_error": (ctypes.c_char_p, []),
+    "kq_version": (_int, []),
+}
+EXPORTED_FUNCTIONS = tuple(_SIGNATURES)
+
+_lib = None
+_lock = threading.Lock()
+
+
+class KroQuantError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str, text: str):
+        super().__init__(f"{fn}: {text} -- {detail}")
+        self.status = status
+
+
+def abi() -> ctypes.CDLL:
+    """The loaded library with argument types set (raises if not built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"KroQuant CUDA library not found at {LIB_PATH}; build it with "
+                        "`python -m w4a4_dit_post_b200.build` (there is no CPU fallback)")
+                lib = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in _SIGNATURES.items():
+                    f = getattr(lib, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = lib
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != KQ_OK:
+        lib = abi()
+        raise KroQuantError(fn, status, lib.kq_last_error().decode(),
+                            lib.kq_status_string(status).decode())
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtypes, ndim: int | None = None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library takes device pointers)")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _x_dtype(x: torch.Tensor) -> int:
+    return KQ_DTYPE_BF16 if x.dtype == torch.bfloat16 else KQ_DTYPE_F32
+
+
+def _out(t, shape, dtype, like, name):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=like.device)
+    _need_cuda(name, t, (dtype,))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, inputs on {like.device}")
+    return t
+
+
+_ACT = (torch.bfloat16, torch.float32)
+
+
+def kq_quantize(x, params, codes=None, scales=None):
+    """KroQuant quantizer: x [M, d] bf16/fp32, params [d/32, 15] fp32 ->
+    (codes uint8 [M, d/2], scales uint8 [M, d/32])."""
+    _need_cuda("x", x, _ACT, 2)
+    _need_cuda("params", params, (torch.float32,))
+    M, d = x.shape
+    codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
+    scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
+    with torch.cuda.device(x.device):
+        _check("kq_quantize", abi().kq_quantize(
+            x.data_ptr(), _x_dtype(x), M, d, params.data_ptr(), codes.data_ptr(),
+            scales.data_ptr(), _stream(x)))
+    return codes, scales
+
+
+def kq_transform(x, params, y=None):
+    """Transform stage alone: y = blockdiag(T_j) x, fp32 [M, d]."""
+    _need_cuda("x", x, _ACT, 2)
+    _need_cuda("params", params, (torch.float32,))
+    M, d = x.shape
+    y = _out(y, (M, d), torch.float32, x, "y")
+    with torch.cuda.device(x.device):
+        _check("kq_transform", abi().kq_transform(
+            x.data_ptr(), _x_dtype(x), M, d, params.data_ptr(), y.data_ptr(), _stream(x)))
+    return y
+
+
+def sq_quantize(x, inv_s, codes=None, scales=None):
+    """SmoothQuant comparison quantizer: y_c = x_c * inv_s[c], then MXFP4."""
+    _need_cuda("x", x, _ACT, 2)
+    _need_cuda("inv_s", inv_s, (torch.float32,), 1)
+    M, d = x.shape
+    codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
+    scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
+    with torch.cuda.device(x.device):
+        _check("sq_quantize", abi().sq_quantize(
+            x.data_ptr(), _x_dtype(x), M, d, inv_s.data_ptr(), codes.data_ptr(),
+            scales.data_ptr(), _stream(x)))
+    return codes, scales
+
+
+def kq_expand_params(params, T=None):
+    """params [nb, 15] -> T [nb, 32, 32] fp32."""
+    _need_cuda("params", params, (torch.float32,))
+    nb = params.numel() // 15
+    T = _out(T, (nb, 32, 32), torch.float32, params, "T")
+    with torch.cuda.device(params.device):
+        _check("kq_expand_params", abi().kq_expand_params(
+            params.data_ptr(), 32 * nb, T.data_ptr(), _stream(params)))
+    return T
+
+
+def kq_fold_weights(W, params, W_out=None):
+    """W [N, d] fp32 -> W blockdiag(T_j)^{-1}.  Pass W_out=W for in place."""
+    _need_cuda("W", W, (torch.float32,), 2)
+    _need_cuda("params", params, (torch.float32,))
+    N, d = W.shape
+    W_out = _out(W_out, (N, d), torch.float32, W, "W_out")
+    with torch.cuda.device(W.device):
+        _check("kq_fold_weights", abi().kq_fold_weights(
+            W.data_ptr(), N, d, params.data_ptr(), W_out.data_ptr(), _stream(W)))
+    return W_out
+
+
+def kq_dequant(codes, scales, out=None):
+    """MXFP4 -> fp32 [M, d]."""
+    _need_cuda("codes", codes, (torch.uint8,), 2)
+    _need_cuda("scales", scales, (torch.uint8,), 2)
+    M, half = codes.shape
+    d = 2 * half
+    if tuple(scales.shape) != (M, d // 32):
+        raise ValueError("scales shape does not match codes")
+    out = _out(out, (M, d), torch.float32, codes, "out")
+    with torch.cuda.device(codes.device):
+        _check("kq_dequant", abi().kq_dequant(
+            codes.data_ptr(), scales.data_ptr(), M, d, out.data_ptr(), _stream(codes)))
+    return out
+
+
+def kq_device_status(device=None, clear: bool = False) -> int:
+    """KQ_DEVSTAT_* bits of a device (synchronises the device)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    flags = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        _check("kq_device_status", abi().kq_device_status(ctypes.byref(flags), int(bool(clear))))
+    return flags.value

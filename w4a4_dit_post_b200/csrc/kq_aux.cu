@@ -1,0 +1,160 @@
+// Support kernels: the dense blocks of the transform (kq_expand_params), the
+// inverse folded into the weights (kq_fold_weights) and MXFP4 decoding
+// (kq_dequant).  None of them is on the per-step path; they are simple,
+// memory-bound grid-stride kernels.
+#include <cuda_runtime.h>
+
+#include "kq.h"
+#include "kq_device.cuh"
+#include "kq_host.h"
+
+namespace kq {
+namespace {
+
+constexpr int kAuxThreads = 256;
+
+// T[j][i][k] = prod_m A_jm[bit(i, 4-m)][bit(k, 4-m)], one thread per entry.
+__global__ void __launch_bounds__(kAuxThreads)
+expand_kernel(const float* __restrict__ params, int nb, float* __restrict__ T) {
+  const int total = nb * 1024;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += gridDim.x * blockDim.x) {
+    const int j = idx >> 10, i = (idx >> 5) & 31, k = idx & 31;
+    const float* p = params + 15 * j;
+    float v = 1.0f;
+#pragma unroll
+    for (int m = 0; m < 5; ++m) {
+      const float4 A = lu_factor(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+      const int bi = (i >> (4 - m)) & 1, bk = (k >> (4 - m)) & 1;
+      const float e = bi ? (bk ? A.w : A.z) : (bk ? A.y : A.x);
+      v = __fmul_rn(v, e);
+    }
+    T[idx] = v;
+  }
+}
+
+// One thread per (weight row, 32-column block): w <- w T_j^{-1}, applied as the
+// butterfly of the transposed inverse factors.  Reads the whole block before
+// writing it, so in-place use is safe.
+__global__ void __launch_bounds__(kAuxThreads)
+fold_kernel(const float* W, const float* __restrict__ params, int nb, int n_blocks, float* W_out) {
+  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n_blocks; g += gridDim.x * blockDim.x) {
+    const int j = g % nb;
+    const float* p = params + 15 * j;
+    float4 B[5];
+#pragma unroll
+    for (int m = 0; m < 5; ++m) B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    const float4* src = reinterpret_cast<const float4*>(W + (size_t)g * 32);
+    float2 v[16];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 t = src[q];
+      v[2 * q] = make_float2(t.x, t.y);
+      v[2 * q + 1] = make_float2(t.z, t.w);
+    }
+    butterfly32(v, B);
+    float4* dst = reinterpret_cast<float4*>(W_out + (size_t)g * 32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      dst[q] = make_float4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
+  }
+}
+
+// E2M1 magnitude of a 3-bit code: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_mag(uint32_t c) {
+  // exponent field e = c >> 1, mantissa bit m = c & 1:
+  // e == 0: m * 0.5 (subnormal); else 2^(e-1) * (1 + m / 2).
+  const uint32_t e = c >> 1, m = c & 1u;
+  if (e == 0) return m ? 0.5f : 0.0f;
+  return __uint_as_float((126u + e) << 23) * (m ? 1.5f : 1.0f);
+}
+
+// One thread per block: 16 code bytes + 1 scale byte -> 32 fp32 values.
+__global__ void __launch_bounds__(kAuxThreads)
+dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int n_blocks,
+               float* __restrict__ out) {
+  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n_blocks; g += gridDim.x * blockDim.x) {
+    const uint4 c = *reinterpret_cast<const uint4*>(codes + (size_t)g * 16);
+    const uint32_t byte = scales[g];
+    // 2^(byte - 127): byte 0 is the subnormal 2^-127, 0xFF is NaN
+    const uint32_t sbits = byte == 255u ? 0x7fc00000u : (byte == 0u ? 0x00400000u : byte << 23);
+    const float s = __uint_as_float(sbits);
+    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+    float4* dst = reinterpret_cast<float4*>(out + (size_t)g * 32);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      float f[8];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const uint32_t nib = (words[w] >> (4 * n)) & 0xFu;
+        const float mag = __fmul_rn(e2m1_mag(nib & 7u), s);
+        f[n] = (nib & 8u) ? -mag : mag;
+      }
+      dst[2 * w] = make_float4(f[0], f[1], f[2], f[3]);
+      dst[2 * w + 1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+  }
+}
+
+int grid_for(int n_items) {
+  int sms = 0;
+  if (sm_count(&sms) != KQ_OK || sms <= 0) sms = 148;
+  const int want = (n_items + kAuxThreads - 1) / kAuxThreads;
+  const int cap = sms * 8;
+  return want < cap ? (want > 0 ? want : 1) : cap;
+}
+
+}  // namespace
+}  // namespace kq
+
+extern "C" {
+
+int kq_expand_params(const float* params, int64_t d, float* T, void* stream) {
+  if (int st = kq::check_shape(1, d, 0, "kq_expand_params")) return st;
+  if (!params || !T) return kq::fail(KQ_ERR_INVALID_ARG, "kq_expand_params: NULL pointer");
+  if (!kq::aligned(params, 4) || !kq::aligned(T, 4))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_expand_params: pointers must be 4-byte aligned");
+  const int64_t nb = d / 32;
+  if (nb > (1 << 20)) return kq::fail(KQ_ERR_UNSUPPORTED, "kq_expand_params: d too large");
+  const int total = (int)(nb * 1024);
+  kq::expand_kernel<<<kq::grid_for(total), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+      params, (int)nb, T);
+  return kq::check_launch("expand_kernel launch");
+}
+
+int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params, float* W_out,
+                    void* stream) {
+  if (int st = kq::check_shape(N, d, 0, "kq_fold_weights")) return st;
+  if (!W || !params || !W_out) return kq::fail(KQ_ERR_INVALID_ARG, "kq_fold_weights: NULL pointer");
+  if (!kq::aligned(W, 16) || !kq::aligned(W_out, 16))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_fold_weights: W and W_out must be 16-byte aligned");
+  if (!kq::aligned(params, 4))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_fold_weights: params must be 4-byte aligned");
+  if (W != W_out) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(W), b = reinterpret_cast<uintptr_t>(W_out);
+    const uintptr_t n = (uintptr_t)(N * d) * sizeof(float);
+    if (a < b + n && b < a + n)
+      return kq::fail(KQ_ERR_INVALID_ARG, "kq_fold_weights: W and W_out overlap partially");
+  }
+  if (N == 0) return KQ_OK;
+  const int nb = (int)(d / 32);
+  const int n_blocks = (int)(N * nb);
+  kq::fold_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+      W, params, nb, n_blocks, W_out);
+  return kq::check_launch("fold_kernel launch");
+}
+
+int kq_dequant(const uint8_t* codes, const uint8_t* scales, int64_t M, int64_t d, float* out,
+               void* stream) {
+  if (int st = kq::check_shape(M, d, 0, "kq_dequant")) return st;
+  if (!codes || !scales || !out) return kq::fail(KQ_ERR_INVALID_ARG, "kq_dequant: NULL pointer");
+  if (!kq::aligned(codes, 16) || !kq::aligned(out, 16))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_dequant: codes and out must be 16-byte aligned");
+  if (M == 0) return KQ_OK;
+  const int n_blocks = (int)(M * (d / 32));
+  kq::dequant_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+      codes, scales, n_blocks, out);
+  return kq::check_launch("dequant_kernel launch");
+}
+
+}  // extern "C"
