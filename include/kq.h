@@ -36,7 +36,8 @@
  *   - arguments are checked on the host before anything is launched; a
  *     non-zero return means nothing was enqueued (KQ_ERR_CUDA: the launch
  *     itself failed; kq_last_error() has the CUDA message);
- *   - M == 0 (or N == 0) is a no-op that returns KQ_OK;
+ *   - M == 0 (or N == 0) is a no-op that returns KQ_OK once the shape and
+ *     dtype are valid; its pointers are not looked at and may be NULL;
  *   - the functions are thread-safe.
  *
  * Device waits.  The streaming kernels wait on shared-memory barriers for

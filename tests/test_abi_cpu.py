@@ -78,6 +78,8 @@ def test_quantize_argument_checks(lib):
     assert q(A16, 0, 4, 32768 + 32, A16b, A16c, A16d, None) == 4   # d limit
     assert q(A16, 0, 2 ** 40, 1024, A16b, A16c, A16d, None) == 4   # block count
     assert q(A16, 0, 0, 64, A16b, A16c, A16d + 1, None) == 0       # M == 0: no-op
+    assert q(None, 0, 0, 64, None, None, None, None) == 0          # ... pointers unused
+    assert q(None, 0, 0, 48, None, None, None, None) == 1          # shape still checked
     assert b"kq_quantize" in lib.kq_last_error()
 
 
@@ -91,6 +93,7 @@ def test_other_argument_checks(lib):
     assert lib.kq_fold_weights(A16, 4, 64, A16b, A16 + 8, None) == 2
     assert lib.kq_fold_weights(A16, 4, 64, A16b, A16 + 64, None) == 1   # partial overlap
     assert lib.kq_fold_weights(A16, 0, 64, A16b, A16c, None) == 0
+    assert lib.kq_fold_weights(None, 0, 64, None, None, None) == 0
     assert lib.kq_dequant(A16, A16b, 4, 64, A16c + 4, None) == 2
     assert lib.kq_dequant(A16, A16b, 0, 64, A16c, None) == 0
     assert lib.kq_device_status(None, 0) == 1

@@ -152,6 +152,23 @@ def test_exact_encoding_identity(kq, scale_pow):
     check(rep, f"identity 2^{scale_pow}")
 
 
+@pytest.mark.parametrize("w", synthetic.workloads(["tiny", "pixart", "sana", "flux"]), ids=lambda w: w.key)
+def test_smoothquant_bit_exact_fp32(kq, w):
+    """SmoothQuant's transform is one multiplication, so the oracle can take
+    every decision in the kernel's precision: y = fl32(x * inv_s) (an IEEE
+    single product in NumPy), then the oracle's MXFP4 encoding.  Codes and
+    scales must match bit for bit, with no exemptions."""
+    xd = device_activations(w)
+    rows = sample_rows(w.M, 512, w.seed)
+    x32 = f64(synthetic.make_activations(w, rows), w.dtype).astype(np.float32)
+    inv_s = synthetic.smoothquant_inv_scales(x32)
+    codes, scales = kq.sq_quantize(xd, torch.from_numpy(inv_s).cuda())
+    y32 = (x32 * inv_s[None, :]).astype(np.float64)
+    c_ref, s_ref = o.quantize_mxfp4(y32)
+    assert np.array_equal(scales[rows].cpu().numpy(), s_ref)
+    assert np.array_equal(codes[rows].cpu().numpy(), c_ref)
+
+
 def test_exact_encoding_smoothquant_unit(kq):
     w = synthetic.Workload("u", 512, 1024, "bf16", "normal", 0.01, None, 100.0, 3.0, 23)
     raw = synthetic.make_activations(w)

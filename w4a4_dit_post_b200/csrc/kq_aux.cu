@@ -125,6 +125,7 @@ int kq_expand_params(const float* params, int64_t d, float* T, void* stream) {
 int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params, float* W_out,
                     void* stream) {
   if (int st = kq::check_shape(N, d, 0, "kq_fold_weights")) return st;
+  if (N == 0) return KQ_OK;
   if (!W || !params || !W_out) return kq::fail(KQ_ERR_INVALID_ARG, "kq_fold_weights: NULL pointer");
   if (!kq::aligned(W, 16) || !kq::aligned(W_out, 16))
     return kq::fail(KQ_ERR_ALIGNMENT, "kq_fold_weights: W and W_out must be 16-byte aligned");
@@ -136,7 +137,6 @@ int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params, f
     if (a < b + n && b < a + n)
       return kq::fail(KQ_ERR_INVALID_ARG, "kq_fold_weights: W and W_out overlap partially");
   }
-  if (N == 0) return KQ_OK;
   const int nb = (int)(d / 32);
   const int n_blocks = (int)(N * nb);
   kq::fold_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
@@ -147,10 +147,10 @@ int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params, f
 int kq_dequant(const uint8_t* codes, const uint8_t* scales, int64_t M, int64_t d, float* out,
                void* stream) {
   if (int st = kq::check_shape(M, d, 0, "kq_dequant")) return st;
+  if (M == 0) return KQ_OK;
   if (!codes || !scales || !out) return kq::fail(KQ_ERR_INVALID_ARG, "kq_dequant: NULL pointer");
   if (!kq::aligned(codes, 16) || !kq::aligned(out, 16))
     return kq::fail(KQ_ERR_ALIGNMENT, "kq_dequant: codes and out must be 16-byte aligned");
-  if (M == 0) return KQ_OK;
   const int n_blocks = (int)(M * (d / 32));
   kq::dequant_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
       codes, scales, n_blocks, out);

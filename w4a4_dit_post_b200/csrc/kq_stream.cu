@@ -321,6 +321,7 @@ int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef
   if (int st = check_shape(M, d, KQ_MAX_D, fn)) return st;
   if (x_dtype != KQ_DTYPE_BF16 && x_dtype != KQ_DTYPE_F32)
     return fail(KQ_ERR_DTYPE, "%s: x_dtype = %d", fn, x_dtype);
+  if (M == 0) return KQ_OK;   // nothing to read or write; pointers may be NULL
   if (!x || !coef) return fail(KQ_ERR_INVALID_ARG, "%s: NULL input pointer", fn);
   if (kOp == Op::kKqTransform) {
     if (!y) return fail(KQ_ERR_INVALID_ARG, "%s: NULL output pointer", fn);
@@ -331,7 +332,6 @@ int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef
   if (!aligned(coef, 4)) return fail(KQ_ERR_ALIGNMENT, "%s: parameters must be 4-byte aligned", fn);
   if (codes && !aligned(codes, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: codes must be 16-byte aligned", fn);
   if (y && !aligned(y, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: y must be 16-byte aligned", fn);
-  if (M == 0) return KQ_OK;
   const cudaStream_t s = as_stream(stream);
   if (x_dtype == KQ_DTYPE_BF16)
     return launch_stream<2, kOp>(x, x_dtype, M, d, coef, codes, scales, y, s);
