@@ -276,17 +276,17 @@ def run_kroquant(args) -> int:
 
     dominant = max(range(len(ws)), key=lambda i: ws[i].M * ws[i].d)
 
-    def one_step(k, fn, ev=None):
+    def one_step(slot, fn, ev=None, ei=0):
         for i, (w, p, inv_s, slots) in enumerate(rings):
-            x, codes, scales = slots[k % R]
+            x, codes, scales = slots[slot % R]
             if ev is not None:
-                ev[i][0][k].record(stream)
+                ev[i][0][ei].record(stream)
             if fn == "kq":
                 kq.kq_quantize(x, p, codes, scales)
             else:
                 kq.sq_quantize(x, inv_s, codes, scales)
             if ev is not None:
-                ev[i][1][k].record(stream)
+                ev[i][1][ei].record(stream)
 
     def timed(fn, K, W, per_launch=False):
         for k in range(W):
@@ -302,7 +302,7 @@ def run_kroquant(args) -> int:
         t0 = time.perf_counter()
         e0.record(stream)
         for k in range(K):
-            one_step(W + k, fn, ev)
+            one_step(W + k, fn, ev, k)
         e1.record(stream)
         torch.cuda.synchronize(device)
         t1 = time.perf_counter()
