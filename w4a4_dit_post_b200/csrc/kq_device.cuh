@@ -7,6 +7,7 @@
 //  * the MXFP4 block encoder (amax, E8M0 byte, E2M1 nibbles).
 #pragma once
 
+#include <cuda_fp4.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -83,6 +84,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
+// Asynchronous 4-byte global -> shared copy (cp.async); all copies a thread
+// issued are awaited with cp_async_wait_all().
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// 3-D tiled TMA load global -> shared (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // element conversion
 // ---------------------------------------------------------------------------
@@ -139,16 +160,35 @@ __device__ __forceinline__ float4 lu_factor_inv_t(float a, float b, float u) {
 // ---------------------------------------------------------------------------
 // MXFP4 encoding of one 32-element block
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float absmax_nan(float a, float b) {
+// max(|a|, |b|) and max(|a|, |b|, |c|), NaN-propagating (a NaN anywhere gives NaN).
+__device__ __forceinline__ float absmax2(float a, float b) {
   float r;
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)));
   return r;
 }
 
-__device__ __forceinline__ float max_nan(float a, float b) {
+__device__ __forceinline__ float absmax3(float a, float b, float c) {
   float r;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
   return r;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Largest magnitude of 32 values: a 3-input max tree of 16 instructions.
+__device__ __forceinline__ float block_absmax(const float2 (&v)[16]) {
+  const float* f = reinterpret_cast<const float*>(v);
+  float m[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) m[i] = absmax3(f[3 * i], f[3 * i + 1], f[3 * i + 2]);
+  m[10] = absmax2(f[30], f[31]);
+  const float q0 = max3(m[0], m[1], m[2]), q1 = max3(m[3], m[4], m[5]);
+  const float q2 = max3(m[6], m[7], m[8]), q3 = max3(m[9], m[10], q0);
+  return max3(q1, q2, q3);
 }
 
 // E8M0 byte of a block with largest magnitude `amax` (NaN if any element is
@@ -167,34 +207,20 @@ __device__ __forceinline__ float inv_scale_from_byte(uint32_t byte) {
 }
 
 // Four pairs -> 8 E2M1 nibbles in one word; element 2i of the pair list lands
-// in nibble 2i (low nibble first).  cvt...e2m1x2 puts its first source in the
-// high nibble, hence the swapped operands.  Rounds to nearest even and
-// saturates to +-6.
+// in nibble 2i (low nibble first).  The conversion is CUDA's own
+// __nv_cvt_float2_to_fp4x2 (round to nearest even, saturating to +-6), which
+// puts x.x in the low nibble of its byte.
 __device__ __forceinline__ uint32_t e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
-      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
-      : "=r"(r)
-      : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x),
-        "f"(p3.y));
-  return r;
+  const uint32_t b0 = __nv_cvt_float2_to_fp4x2(p0, __NV_E2M1, cudaRoundNearest);
+  const uint32_t b1 = __nv_cvt_float2_to_fp4x2(p1, __NV_E2M1, cudaRoundNearest);
+  const uint32_t b2 = __nv_cvt_float2_to_fp4x2(p2, __NV_E2M1, cudaRoundNearest);
+  const uint32_t b3 = __nv_cvt_float2_to_fp4x2(p3, __NV_E2M1, cudaRoundNearest);
+  return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
 }
 
 // Encode 32 values: returns the scale byte and writes 16 code bytes to `out`.
 __device__ __forceinline__ uint32_t mxfp4_encode32(const float2 (&v)[16], uint4& out) {
-  float m[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    m[i] = max_nan(absmax_nan(v[2 * i].x, v[2 * i].y), absmax_nan(v[2 * i + 1].x, v[2 * i + 1].y));
-#pragma unroll
-  for (int s = 4; s >= 1; s >>= 1)
-#pragma unroll
-    for (int i = 0; i < s; ++i) m[i] = max_nan(m[i], m[i + s]);
-  const uint32_t byte = e8m0_byte(m[0]);
+  const uint32_t byte = e8m0_byte(block_absmax(v));
   const float sc = inv_scale_from_byte(byte);
   const float2 sc2 = make_float2(sc, sc);
   float2 r[16];

@@ -1,26 +1,37 @@
 // Streaming kernels of the online quantizer: kq_quantize, kq_transform and
 // the SmoothQuant comparison quantizer sq_quantize.
 //
-// Data view.  Rows are contiguous and d is a multiple of 32, so an [M][d]
-// activation is a flat array of M*d/32 blocks of 32 elements; block g is
-// token g / nb, channel block j = g % nb.  Its 16 code bytes sit at
-// codes + 16 g and its scale byte at scales + g, so one thread per block
-// writes coalesced 16-byte and 1-byte stores.
+// Tiling.  An activation [M][d] is viewed as [M rows][nb blocks][32 elements]
+// (rows contiguous, nb = d / 32).  The nb block columns are cut into NC
+// column groups of C consecutive blocks (C = the largest divisor of nb not
+// above 32) and the rows into row tiles of R rows, R = 2 * floor(256 / C).  A
+// tile (R x C blocks, at most 32 KiB of bf16) arrives in shared memory by one
+// 3-D TMA load (box 32 x C x R, 64-byte swizzle for bf16 rows, 128-byte for
+// fp32 rows); the swizzle makes each thread's 16-byte reads of a whole block
+// conflict-free.
 //
-// Pipeline.  A persistent grid (a whole number of CTAs per SM); each CTA
-// walks tiles of 256 blocks (one per thread).  Thread 0 keeps kStages tiles
-// in flight with 2-D TMA loads (box = 32 elements x 256 blocks) into
-// swizzled shared memory, each stage guarded by an mbarrier.  The swizzle
-// (64-byte for bf16 rows, 128-byte for fp32 rows) makes the per-thread
-// 16-byte reads of a whole 64/128-byte block conflict-free.  After reading
-// its block into registers a thread joins a CTA barrier, and thread 0 reuses
-// the stage for the tile kStages ahead; the transform, the encoding and the
-// stores then overlap the loads in flight.
+// Column-stationary persistent grid.  The grid is a multiple of NC; CTA b owns
+// column group b % NC for its whole life and walks every (G / NC)-th row
+// tile.  Its transform coefficients therefore cover only C block columns and
+// are built once, in a small shared table.  Thread t owns block column
+// t % C and the row pair (2 (t / C), 2 (t / C) + 1) of every tile: the two
+// rows share their coefficients, so every butterfly operation is one packed
+// f32x2 instruction on (row 0, row 1) with a broadcast coefficient.
 //
-// Per-block coefficients are built once per CTA in shared memory: for
-// KroQuant 5 factors x (A00, A01, A10, A11) from the 15 LU parameters; for
-// SmoothQuant the 32 inverse scales.  Row strides of 80 and 144 bytes (5 and
-// 9 16-byte units, odd) keep 8 consecutive blocks on distinct bank groups.
+// Transform.  Each LU factor A = L U (L = [[1,0],[a,1]], U = [[u,b],[0,1/u]])
+// is split as A = S L'' U' with S = diag(u, 1/u), U' = [[1, b/u], [0, 1]] and
+// L'' = [[1, 0], [a u^2, 1]].  The diagonal S of one Kronecker position
+// commutes with the factors at the other positions, so
+//     T = (x)_m A_m = D (x)_m L''_m (x)_m U'_m,   D = (x)_m S_m (diagonal),
+// and the block transform is ten shear passes (one FMA per element pair
+// each) and one diagonal scaling: 6 flops per element instead of 10.  The
+// sizes of the summed terms are unchanged: D |L''| |U'| = |L| |U| entrywise.
+//
+// Pipeline.  Thread 0 keeps kStages tiles in flight; each stage is guarded by
+// an mbarrier (bounded waits).  After copying its two blocks into registers
+// a thread joins a CTA barrier, thread 0 reuses the stage for the tile
+// kStages ahead, and the transform, the MXFP4 encoding and the stores
+// overlap the loads in flight.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -38,89 +49,209 @@ namespace kq {
 __device__ unsigned int g_devstat = 0;
 
 constexpr int kThreads = 256;
-constexpr int kTileBlocks = 256;   // blocks per tile = TMA box rows
+constexpr int kMaxC = 32;
 
 enum class Op : int { kKqQuant = 0, kKqTransform = 1, kSqQuant = 2 };
+
+// Tile geometry, computed on the host and passed by value.
+struct Geometry {
+  int nb;           // blocks per row
+  int C;            // blocks per column group
+  int NC;           // column groups
+  int R;            // rows per tile
+  int M;            // rows
+  int n_row_tiles;
+  int stage_bytes;  // R * C * block bytes, rounded up to 1024
+};
 
 template <int kInBytes>
 struct InLayout;
 
 template <>
-struct InLayout<2> {                     // bf16: 64-byte block rows, 64B swizzle
+struct InLayout<2> {                     // bf16: 64-byte blocks, 64B swizzle
   static constexpr int kBlockBytes = 64;
-  static constexpr int kChunks = 4;      // 16-byte chunks per block
-  __device__ static int swz(int t) { return (t >> 1) & 3; }
+  // physical 16-byte chunk of logical chunk q in shared block-row b
+  __device__ static int chunk(int b, int q) { return q ^ ((b >> 1) & 3); }
 };
 
 template <>
-struct InLayout<4> {                     // fp32: 128-byte block rows, 128B swizzle
+struct InLayout<4> {                     // fp32: 128-byte blocks, 128B swizzle
   static constexpr int kBlockBytes = 128;
-  static constexpr int kChunks = 8;
-  __device__ static int swz(int t) { return t & 7; }
+  __device__ static int chunk(int b, int q) { return q ^ (b & 7); }
 };
 
+// Coefficient table row per block column (floats).  KroQuant: ten shear
+// coefficients and 32 diagonal entries, each stored twice (the packed pair
+// of a broadcast operand): 84 floats, 21 16-byte units (odd, so 8 threads
+// on consecutive columns hit distinct bank groups).  SmoothQuant: the 32
+// inverse scales, each stored twice, padded to 68 floats (17 units).
 template <Op kOp>
-struct TableLayout {
-  // floats per coefficient row (padded to an odd number of 16-byte units)
-  static constexpr int kRowFloats = (kOp == Op::kSqQuant) ? 36 : 20;
-};
-
-template <int kInBytes, Op kOp>
-struct StreamCfg {
-  static constexpr int kStages = (kInBytes == 2) ? 4 : 2;
-  static constexpr int kStageBytes = kTileBlocks * InLayout<kInBytes>::kBlockBytes;
-  static constexpr int kBarOffset = kStages * kStageBytes;
-  static constexpr int kTableOffset = kBarOffset + 128;
-  static size_t smem_bytes(int nb) {
-    // + 1024 for aligning the dynamic base to the 1024-byte swizzle atom
-    return 1024 + kTableOffset + (size_t)nb * TableLayout<kOp>::kRowFloats * sizeof(float);
-  }
+struct Table {
+  static constexpr int kRowFloats = (kOp == Op::kSqQuant) ? 68 : 84;
 };
 
 template <int kInBytes>
-__device__ __forceinline__ void load_block(const uint8_t* stage, int tid, float2 (&v)[16]) {
+struct StageCfg {
+  static constexpr int kStages = (kInBytes == 2) ? 3 : 2;
+};
+
+// Largest divisor of nb that is at most kMaxC.
+inline int choose_C(int nb) {
+  for (int c = nb < kMaxC ? nb : kMaxC; c > 1; --c)
+    if (nb % c == 0) return c;
+  return 1;
+}
+
+template <int kInBytes>
+inline Geometry make_geometry(int64_t M, int nb) {
+  Geometry g;
+  g.nb = nb;
+  g.C = choose_C(nb);
+  g.NC = nb / g.C;
+  int R = 2 * (kThreads / g.C);
+  if (R > 256) R = 256;                  // TMA box dimension limit
+  g.R = R;
+  g.M = (int)M;
+  g.n_row_tiles = (int)((M + R - 1) / R);
+  const int raw = R * g.C * InLayout<kInBytes>::kBlockBytes;
+  g.stage_bytes = (raw + 1023) & ~1023;
+  return g;
+}
+
+template <int kInBytes, Op kOp>
+inline size_t smem_bytes(const Geometry& g) {
+  // + staging for the raw coefficients: C * 32 floats
+  return 1024 /* base alignment */ + (size_t)StageCfg<kInBytes>::kStages * g.stage_bytes + 128 +
+         (size_t)g.C * (Table<kOp>::kRowFloats + 32) * sizeof(float);
+}
+
+// Two blocks (rows 2 rp and 2 rp + 1 of block column c of a tile) from a
+// stage, as 32 packed pairs v[i] = (first row element i, second row element i).
+template <int kInBytes>
+__device__ __forceinline__ void load_pair(const uint8_t* stage, int C, int rp, int c,
+                                          float2 (&v)[32]) {
   using L = InLayout<kInBytes>;
-  const uint8_t* row = stage + tid * L::kBlockBytes;
-  const int sw = L::swz(tid);
-  uint4 q[L::kChunks];
-#pragma unroll
-  for (int c = 0; c < L::kChunks; ++c)
-    q[c] = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+  const int b0 = (2 * rp) * C + c, b1 = b0 + C;
+  const uint8_t* p0 = stage + b0 * L::kBlockBytes;
+  const uint8_t* p1 = stage + b1 * L::kBlockBytes;
   if constexpr (kInBytes == 2) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      v[4 * c + 0] = bf16x2_to_float2(q[c].x);
-      v[4 * c + 1] = bf16x2_to_float2(q[c].y);
-      v[4 * c + 2] = bf16x2_to_float2(q[c].z);
-      v[4 * c + 3] = bf16x2_to_float2(q[c].w);
+    for (int q = 0; q < 4; ++q) {
+      const uint4 w0 = *reinterpret_cast<const uint4*>(p0 + (L::chunk(b0, q) << 4));
+      const uint4 w1 = *reinterpret_cast<const uint4*>(p1 + (L::chunk(b1, q) << 4));
+      const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w};
+      const uint32_t a1[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {  // word e of chunk q holds elements 8q+2e, 8q+2e+1
+        v[8 * q + 2 * e] = make_float2(__uint_as_float(a0[e] << 16), __uint_as_float(a1[e] << 16));
+        v[8 * q + 2 * e + 1] = make_float2(__uint_as_float(a0[e] & 0xffff0000u),
+                                           __uint_as_float(a1[e] & 0xffff0000u));
+      }
     }
   } else {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      v[2 * c + 0] = make_float2(__uint_as_float(q[c].x), __uint_as_float(q[c].y));
-      v[2 * c + 1] = make_float2(__uint_as_float(q[c].z), __uint_as_float(q[c].w));
+    for (int q = 0; q < 8; ++q) {
+      const float4 w0 = *reinterpret_cast<const float4*>(p0 + (L::chunk(b0, q) << 4));
+      const float4 w1 = *reinterpret_cast<const float4*>(p1 + (L::chunk(b1, q) << 4));
+      v[4 * q + 0] = make_float2(w0.x, w1.x);
+      v[4 * q + 1] = make_float2(w0.y, w1.y);
+      v[4 * q + 2] = make_float2(w0.z, w1.z);
+      v[4 * q + 3] = make_float2(w0.w, w1.w);
     }
   }
+}
+
+// KroQuant transform of a row pair from one coefficient row.  Row layout:
+// floats [4m .. 4m+3] = (b_m/u_m, b_m/u_m, a_m u_m^2, a_m u_m^2) for m = 0..4,
+// then [20 + 2i], [21 + 2i] = D_i twice for i = 0..31.
+__device__ __forceinline__ void kq_transform_pair(float2 (&v)[32], const float* row) {
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+#pragma unroll
+  for (int m = 0; m < 5; ++m) {
+    const int h = 1 << (4 - m);             // factor m acts on element-index bit 4 - m
+    const float4 sh = r4[m];
+    const float2 beta = make_float2(sh.x, sh.y), gamma = make_float2(sh.z, sh.w);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i & h) continue;
+      v[i] = __ffma2_rn(beta, v[i + h], v[i]);        // U':  lo += (b/u) hi
+      v[i + h] = __ffma2_rn(gamma, v[i], v[i + h]);   // L'':  hi += (a u^2) lo
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const float4 dd = r4[5 + q];            // (D_2q, D_2q, D_2q+1, D_2q+1)
+    v[2 * q] = __fmul2_rn(v[2 * q], make_float2(dd.x, dd.y));
+    v[2 * q + 1] = __fmul2_rn(v[2 * q + 1], make_float2(dd.z, dd.w));
+  }
+}
+
+__device__ __forceinline__ void sq_transform_pair(float2 (&v)[32], const float* row) {
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const float4 s = r4[q];
+    v[2 * q] = __fmul2_rn(v[2 * q], make_float2(s.x, s.y));
+    v[2 * q + 1] = __fmul2_rn(v[2 * q + 1], make_float2(s.z, s.w));
+  }
+}
+
+template <int kSel>
+__device__ __forceinline__ float lane(const float2& p) {
+  return kSel ? p.y : p.x;
+}
+
+// Largest magnitude of lane kSel (0: first row, 1: second), NaN-propagating.
+template <int kSel>
+__device__ __forceinline__ float lane_absmax(const float2 (&v)[32]) {
+  float m[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i)
+    m[i] = absmax3(lane<kSel>(v[3 * i]), lane<kSel>(v[3 * i + 1]), lane<kSel>(v[3 * i + 2]));
+  m[10] = absmax2(lane<kSel>(v[30]), lane<kSel>(v[31]));
+  const float q0 = max3(m[0], m[1], m[2]), q1 = max3(m[3], m[4], m[5]);
+  const float q2 = max3(m[6], m[7], m[8]), q3 = max3(m[9], m[10], q0);
+  return max3(q1, q2, q3);
+}
+
+// E2M1 codes of lane kSel: 16 bytes, element 2k in the low nibble of byte k.
+template <int kSel>
+__device__ __forceinline__ uint4 lane_codes(const float2 (&r)[32]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int b = 8 * q;
+    w[q] = e2m1x8(make_float2(lane<kSel>(r[b]), lane<kSel>(r[b + 1])),
+                  make_float2(lane<kSel>(r[b + 2]), lane<kSel>(r[b + 3])),
+                  make_float2(lane<kSel>(r[b + 4]), lane<kSel>(r[b + 5])),
+                  make_float2(lane<kSel>(r[b + 6]), lane<kSel>(r[b + 7])));
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 template <int kInBytes, Op kOp>
 __global__ void __launch_bounds__(kThreads, 2)
 stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ coef_src,
-              int nb, int n_blocks, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+              const Geometry geo, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
               float* __restrict__ y_out) {
-  using Cfg = StreamCfg<kInBytes, kOp>;
-  constexpr int kStages = Cfg::kStages;
-  constexpr int kRow = TableLayout<kOp>::kRowFloats;
+  constexpr int kStages = StageCfg<kInBytes>::kStages;
+  constexpr int kRow = Table<kOp>::kRowFloats;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);
-  int* abort_flag = reinterpret_cast<int*>(smem + Cfg::kBarOffset + 8 * kStages);
-  float* table = reinterpret_cast<float*>(smem + Cfg::kTableOffset);
+  const int stage_bytes = geo.stage_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes);
+  int* abort_flag = reinterpret_cast<int*>(smem + kStages * stage_bytes + 8 * kStages);
+  float* table = reinterpret_cast<float*>(smem + kStages * stage_bytes + 128);
 
   const int tid = threadIdx.x;
-  const int n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
+  const int C = geo.C, R = geo.R;
+  const int col_group = blockIdx.x % geo.NC;
+  const int row_step = gridDim.x / geo.NC;      // CTAs sharing this column group
+  const int rt_first = blockIdx.x / geo.NC;
+  const int j0 = col_group * C;                 // first block column of the group
+  const uint32_t tile_tx = (uint32_t)(R * C * InLayout<kInBytes>::kBlockBytes);
 
   if (tid == 0) {
     tma_prefetch_desc(&tmap);
@@ -133,96 +264,124 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   if (tid == 0) {
 #pragma unroll
     for (int s = 0; s < kStages; ++s) {
-      const int tile = blockIdx.x + s * gridDim.x;
-      if (tile < n_tiles) {
-        mbar_arrive_expect_tx(smem_addr(&bars[s]), Cfg::kStageBytes);
-        tma_load_2d(smem_addr(smem + s * Cfg::kStageBytes), &tmap, 0, tile * kTileBlocks,
-                    smem_addr(&bars[s]));
+      const int rt = rt_first + s * row_step;
+      if (rt < geo.n_row_tiles) {
+        mbar_arrive_expect_tx(smem_addr(&bars[s]), tile_tx);
+        tma_load_3d(smem_addr(smem + s * stage_bytes), &tmap, 0, j0, rt * R, smem_addr(&bars[s]));
       }
     }
   }
 
-  // coefficient table (overlaps the first loads)
+  // Coefficients of this CTA's C block columns, overlapping the first loads.
+  // The raw parameters are staged with asynchronous copies (all in flight at
+  // once: one memory round trip), then turned into table rows from shared
+  // memory only.
   if constexpr (kOp == Op::kSqQuant) {
-    for (int i = tid; i < nb * 32; i += kThreads)
-      table[(i >> 5) * kRow + (i & 31)] = coef_src[i];
+    float* stage_in = table + C * kRow;                 // C * 32 inverse scales
+    for (int i = tid; i < C * 32; i += kThreads) cp_async_4(smem_addr(stage_in + i), coef_src + 32 * j0 + i);
+    cp_async_wait_all();
+    __syncthreads();
+    for (int i = tid; i < C * 32; i += kThreads) {
+      const float sv = stage_in[i];
+      *reinterpret_cast<float2*>(table + (i >> 5) * kRow + 2 * (i & 31)) = make_float2(sv, sv);
+    }
   } else {
-    for (int i = tid; i < nb * 5; i += kThreads) {
-      const int j = i / 5, m = i - 5 * j;
-      const float* p = coef_src + 15 * j + 3 * m;
-      *reinterpret_cast<float4*>(table + j * kRow + 4 * m) = lu_factor(p[0], p[1], p[2]);
+    float* prm = table + C * kRow;                      // C * 15 parameters
+    float* uu = prm + C * 16;                           // C * 10: (u_m, 1/u_m)
+    for (int i = tid; i < C * 15; i += kThreads) cp_async_4(smem_addr(prm + i), coef_src + 15 * j0 + i);
+    cp_async_wait_all();
+    __syncthreads();
+    // thread (c, m): the two shears of factor m and (u, 1/u)
+    for (int i = tid; i < C * 5; i += kThreads) {
+      const int cc = i / 5, m = i - 5 * cc;
+      const float a = prm[15 * cc + 3 * m], b = prm[15 * cc + 3 * m + 1], u = prm[15 * cc + 3 * m + 2];
+      const float beta = b / u, gamma = __fmul_rn(__fmul_rn(a, u), u);
+      *reinterpret_cast<float4*>(table + cc * kRow + 4 * m) = make_float4(beta, beta, gamma, gamma);
+      uu[10 * cc + 2 * m] = u;
+      uu[10 * cc + 2 * m + 1] = 1.0f / u;
+    }
+    __syncthreads();
+    // thread (c, e): D_e = prod_m (bit (4 - m) of e ? 1/u_m : u_m)
+    for (int i = tid; i < C * 32; i += kThreads) {
+      const int cc = i >> 5, e = i & 31;
+      float dval = 1.0f;
+#pragma unroll
+      for (int m = 0; m < 5; ++m) dval = __fmul_rn(dval, uu[10 * cc + 2 * m + ((e >> (4 - m)) & 1)]);
+      *reinterpret_cast<float2*>(table + cc * kRow + 20 + 2 * e) = make_float2(dval, dval);
     }
   }
   __syncthreads();
 
-  const int step = kTileBlocks * gridDim.x;       // blocks between a thread's tiles
-  const int jstep = step % nb;
-  int j = (blockIdx.x * kTileBlocks + tid) % nb;  // channel block of this thread's block
+  const int c = tid % C, rp = tid / C;
+  const bool active = rp < R / 2;
+  const float* crow = table + c * kRow;
+  const int nb = geo.nb;
 
   int k = 0;
-  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++k) {
+  for (int rt = rt_first; rt < geo.n_row_tiles; rt += row_step, ++k) {
     const int s = k % kStages;
     const uint32_t parity = (uint32_t)(k / kStages) & 1u;
-    const uint8_t* stage = smem + s * Cfg::kStageBytes;
-    float2 v[16];
+    float2 v[32];
     const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity);
     if (ok) {
-      load_block<kInBytes>(stage, tid, v);
+      if (active) load_pair<kInBytes>(smem + s * stage_bytes, C, rp, c, v);
     } else {
       *abort_flag = 1;
       atomicOr(&g_devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
     }
     __syncthreads();
     if (*abort_flag) {
-      // Give the loads still in flight (tiles k .. k + kStages - 1) time to land
-      // before the CTA's shared memory goes away, then stop.
+      // let the loads still in flight land before shared memory goes away
       if (tid == 0) {
         for (int kk = k; kk < k + kStages; ++kk) {
-          if (blockIdx.x + kk * gridDim.x >= n_tiles) break;
+          if (rt_first + kk * row_step >= geo.n_row_tiles) break;
           (void)mbar_wait_bounded(smem_addr(&bars[kk % kStages]), (uint32_t)(kk / kStages) & 1u);
         }
       }
       return;
     }
     if (tid == 0) {
-      const int nt = tile + kStages * gridDim.x;
-      if (nt < n_tiles) {
-        mbar_arrive_expect_tx(smem_addr(&bars[s]), Cfg::kStageBytes);
-        tma_load_2d(smem_addr(smem + s * Cfg::kStageBytes), &tmap, 0, nt * kTileBlocks,
-                    smem_addr(&bars[s]));
+      const int nrt = rt + kStages * row_step;
+      if (nrt < geo.n_row_tiles) {
+        mbar_arrive_expect_tx(smem_addr(&bars[s]), tile_tx);
+        tma_load_3d(smem_addr(smem + s * stage_bytes), &tmap, 0, j0, nrt * R, smem_addr(&bars[s]));
       }
+    }
+    if (!active) continue;
+
+    const int r0 = rt * R + 2 * rp;             // rows r0 and r0 + 1
+    if (r0 >= geo.M) continue;
+    const bool second = r0 + 1 < geo.M;
+    const size_t g0 = (size_t)r0 * nb + j0 + c; // flat block index of (r0, column)
+
+    if constexpr (kOp == Op::kSqQuant) {
+      sq_transform_pair(v, crow);
+    } else {
+      kq_transform_pair(v, crow);
     }
 
-    const int g = tile * kTileBlocks + tid;
-    if (g < n_blocks) {
-      const float* crow = table + j * kRow;
-      if constexpr (kOp == Op::kSqQuant) {
+    if constexpr (kOp == Op::kKqTransform) {
+      float4* d0 = reinterpret_cast<float4*>(y_out + g0 * 32);
+      float4* d1 = reinterpret_cast<float4*>(y_out + (g0 + nb) * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 c = *reinterpret_cast<const float4*>(crow + 4 * q);
-          v[2 * q + 0] = __fmul2_rn(v[2 * q + 0], make_float2(c.x, c.y));
-          v[2 * q + 1] = __fmul2_rn(v[2 * q + 1], make_float2(c.z, c.w));
-        }
-      } else {
-        float4 A[5];
-#pragma unroll
-        for (int m = 0; m < 5; ++m) A[m] = *reinterpret_cast<const float4*>(crow + 4 * m);
-        butterfly32(v, A);
+      for (int q = 0; q < 8; ++q) {
+        d0[q] = make_float4(v[4 * q].x, v[4 * q + 1].x, v[4 * q + 2].x, v[4 * q + 3].x);
+        if (second)
+          d1[q] = make_float4(v[4 * q].y, v[4 * q + 1].y, v[4 * q + 2].y, v[4 * q + 3].y);
       }
-      if constexpr (kOp == Op::kKqTransform) {
-        float4* dst = reinterpret_cast<float4*>(y_out + (size_t)g * 32);
+    } else {
+      const uint32_t e0 = e8m0_byte(lane_absmax<0>(v));
+      const uint32_t e1 = e8m0_byte(lane_absmax<1>(v));
+      const float2 sc = make_float2(inv_scale_from_byte(e0), inv_scale_from_byte(e1));
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          dst[q] = make_float4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
-      } else {
-        uint4 packed;
-        const uint32_t byte = mxfp4_encode32(v, packed);
-        *reinterpret_cast<uint4*>(codes + (size_t)g * 16) = packed;
-        scales[g] = (uint8_t)byte;
+      for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], sc);
+      *reinterpret_cast<uint4*>(codes + g0 * 16) = lane_codes<0>(v);
+      scales[g0] = (uint8_t)e0;
+      if (second) {
+        *reinterpret_cast<uint4*>(codes + (g0 + nb) * 16) = lane_codes<1>(v);
+        scales[g0 + nb] = (uint8_t)e1;
       }
     }
-    j += jstep;
-    if (j >= nb) j -= nb;
   }
 }
 
@@ -252,20 +411,20 @@ int get_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
   return KQ_OK;
 }
 
-// Tensor map over the flat block view: dim0 = 32 elements, dim1 = n_blocks.
-int make_block_tmap(CUtensorMap* tm, const void* x, int x_dtype, int n_blocks) {
+// Tensor map over [M][nb][32]: box = 32 elements x C blocks x R rows.
+template <int kInBytes>
+int make_tile_tmap(CUtensorMap* tm, const void* x, const Geometry& g) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   if (int st = get_encoder(&enc)) return st;
-  const bool bf16 = (x_dtype == KQ_DTYPE_BF16);
-  const cuuint64_t dims[2] = {32, (cuuint64_t)n_blocks};
-  const cuuint64_t strides[1] = {(cuuint64_t)(bf16 ? 64 : 128)};
-  const cuuint32_t box[2] = {32, (cuuint32_t)kTileBlocks};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                         2, const_cast<void*>(x), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const cuuint64_t dims[3] = {32, (cuuint64_t)g.nb, (cuuint64_t)g.M};
+  const cuuint64_t strides[2] = {(cuuint64_t)(32 * kInBytes), (cuuint64_t)g.nb * 32 * kInBytes};
+  const cuuint32_t box[3] = {32, (cuuint32_t)g.C, (cuuint32_t)g.R};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      enc(tm, kInBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+          const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          kInBytes == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return KQ_OK;
 }
@@ -273,29 +432,25 @@ int make_block_tmap(CUtensorMap* tm, const void* x, int x_dtype, int n_blocks) {
 constexpr int kMaxDevices = 64;
 
 template <int kInBytes, Op kOp>
-int launch_stream(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef,
-                  uint8_t* codes, uint8_t* scales, float* y, cudaStream_t stream) {
-  using Cfg = StreamCfg<kInBytes, kOp>;
+int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_t* codes,
+                  uint8_t* scales, float* y, cudaStream_t stream) {
   const int nb = (int)(d / 32);
-  const int n_blocks = (int)(M * nb);
+  const Geometry geo = make_geometry<kInBytes>(M, nb);
   auto kern = stream_kernel<kInBytes, kOp>;
-  const size_t smem = Cfg::smem_bytes(nb);
+  const size_t smem = smem_bytes<kInBytes, kOp>(geo);
 
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
-  // per-device, per-instantiation: raise the dynamic shared memory limit once
+  if (dev < 0 || dev >= kMaxDevices) return fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  // per device and instantiation: allow the largest dynamic shared memory once
   static std::once_flag attr_once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
-  if (dev < 0 || dev >= kMaxDevices) return fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
   std::call_once(attr_once[dev], [&] {
     int optin = 0;
     attr_err[dev] = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (attr_err[dev] == cudaSuccess) {
-      size_t want = Cfg::smem_bytes(KQ_MAX_D / 32);
-      if (want > (size_t)optin) want = (size_t)optin;
-      attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want);
-    }
+    if (attr_err[dev] == cudaSuccess)
+      attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
 
@@ -307,11 +462,14 @@ int launch_stream(const void* x, int x_dtype, int64_t M, int64_t d, const float*
   if (per_sm < 1) return fail(KQ_ERR_UNSUPPORTED, "kernel does not fit on an SM (smem %zu)", smem);
 
   CUtensorMap tm;
-  if (int st = make_block_tmap(&tm, x, x_dtype, n_blocks)) return st;
-  const int n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
-  int grid = sms * per_sm;
-  if (grid > n_tiles) grid = n_tiles;
-  kern<<<grid, kThreads, smem, stream>>>(tm, coef, nb, n_blocks, codes, scales, y);
+  if (int st = make_tile_tmap<kInBytes>(&tm, x, geo)) return st;
+  // a whole number of CTAs per column group, no more than there are row tiles
+  const int64_t slots = (int64_t)sms * per_sm;
+  int64_t per_group = slots / geo.NC;
+  if (per_group < 1) per_group = 1;
+  if (per_group > geo.n_row_tiles) per_group = geo.n_row_tiles;
+  const int64_t grid = per_group * geo.NC;
+  kern<<<(unsigned)grid, kThreads, smem, stream>>>(tm, coef, geo, codes, scales, y);
   return check_launch("stream_kernel launch");
 }
 
@@ -333,9 +491,8 @@ int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef
   if (codes && !aligned(codes, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: codes must be 16-byte aligned", fn);
   if (y && !aligned(y, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: y must be 16-byte aligned", fn);
   const cudaStream_t s = as_stream(stream);
-  if (x_dtype == KQ_DTYPE_BF16)
-    return launch_stream<2, kOp>(x, x_dtype, M, d, coef, codes, scales, y, s);
-  return launch_stream<4, kOp>(x, x_dtype, M, d, coef, codes, scales, y, s);
+  if (x_dtype == KQ_DTYPE_BF16) return launch_stream<2, kOp>(x, M, d, coef, codes, scales, y, s);
+  return launch_stream<4, kOp>(x, M, d, coef, codes, scales, y, s);
 }
 
 }  // namespace
