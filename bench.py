@@ -73,9 +73,12 @@ def step_bytes(ws) -> float:
     return sum(algorithmic_bytes(w.M, w.d) for w in ws)
 
 
-def ring_depth(ws, l2_bytes: int) -> int:
-    per_step = sum(w.M * w.d * (2 + 0.5 + 1 / 32) for w in ws)
-    return max(2, int(math.ceil(RING_FACTOR_L2 * l2_bytes / per_step)))
+def ring_depth(w, l2_bytes: int) -> int:
+    """Distinct input/output buffer sets for shape w so that cycling through
+    them touches more than RING_FACTOR_L2 times the L2 size (every launch,
+    including back-to-back launches of one shape, reads cold data)."""
+    per_launch = w.M * w.d * (2 + 0.5 + 1 / 32)
+    return max(2, int(math.ceil(RING_FACTOR_L2 * l2_bytes / per_launch)))
 
 
 # ---------------------------------------------------------------------------
@@ -247,7 +250,7 @@ def run_kroquant(args) -> int:
     l2 = int(getattr(props, "L2_cache_size", 0) or 126 * 2 ** 20)
 
     ws = step_workloads(rank)
-    R = ring_depth(ws, l2)
+    Rs = [ring_depth(w, l2) for w in ws]
     stream = torch.cuda.current_stream(device)
 
     # inputs: the seeded workload, then R-1 row rotations of it (distinct buffers)
@@ -264,7 +267,7 @@ def run_kroquant(args) -> int:
         inv_s = torch.from_numpy(synthetic.smoothquant_inv_scales(
             synthetic.f32_from_bf16_bits(raw[:: max(1, w.M // 1024)]))).to(device)
         slots = []
-        for r in range(R):
+        for r in range(ring_depth(w, l2)):
             x = x0 if r == 0 else torch.roll(x0, shifts=r * 997, dims=0).contiguous()
             codes = torch.empty((w.M, w.d // 2), dtype=torch.uint8, device=device)
             scales = torch.empty((w.M, w.d // 32), dtype=torch.uint8, device=device)
@@ -276,25 +279,23 @@ def run_kroquant(args) -> int:
 
     dominant = max(range(len(ws)), key=lambda i: ws[i].M * ws[i].d)
 
-    def one_step(slot, fn, ev=None, ei=0):
-        for i, (w, p, inv_s, slots) in enumerate(rings):
-            x, codes, scales = slots[slot % R]
-            if ev is not None:
-                ev[i][0][ei].record(stream)
-            if fn == "kq":
-                kq.kq_quantize(x, p, codes, scales)
-            else:
-                kq.sq_quantize(x, inv_s, codes, scales)
-            if ev is not None:
-                ev[i][1][ei].record(stream)
+    def launch(i, slot, fn):
+        w, p, inv_s, slots = rings[i]
+        x, codes, scales = slots[slot % len(slots)]
+        if fn == "kq":
+            kq.kq_quantize(x, p, codes, scales)
+        elif fn == "tc":
+            kq.kq_quantize_tc(x, p, codes, scales)
+        else:
+            kq.sq_quantize(x, inv_s, codes, scales)
 
-    def timed(fn, K, W, per_launch=False):
+    def timed_steps(fn, K, W):
+        """K whole steps (every shape once) between two events; no events in
+        between, so consecutive launches may overlap their launch latency
+        (programmatic dependent launch)."""
         for k in range(W):
-            one_step(k, fn)
-        ev = None
-        if per_launch:
-            ev = [([torch.cuda.Event(enable_timing=True) for _ in range(K)],
-                   [torch.cuda.Event(enable_timing=True) for _ in range(K)]) for _ in rings]
+            for i in range(len(rings)):
+                launch(i, k, fn)
         barrier(world, device)
         torch.cuda.synchronize(device)
         e0 = torch.cuda.Event(enable_timing=True)
@@ -302,43 +303,51 @@ def run_kroquant(args) -> int:
         t0 = time.perf_counter()
         e0.record(stream)
         for k in range(K):
-            one_step(W + k, fn, ev, k)
+            for i in range(len(rings)):
+                launch(i, W + k, fn)
         e1.record(stream)
         torch.cuda.synchronize(device)
         t1 = time.perf_counter()
         barrier(world, device)
-        ms = e0.elapsed_time(e1)
-        launch_ms = None
-        if per_launch:
-            launch_ms = [sum(a.elapsed_time(b) for a, b in zip(ev[i][0], ev[i][1])) / K
-                         for i in range(len(rings))]
-        return ms, launch_ms, t0, t1
+        return e0.elapsed_time(e1), t0, t1
+
+    def timed_burst(i, fn, K, W):
+        """Average device time of one launch of shape i: K back-to-back
+        launches of that shape (cycling the ring) between two events."""
+        for k in range(W):
+            launch(i, k, fn)
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(K):
+            launch(i, W + k, fn)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / K
 
     K, W = args.steps, args.warmup
     if args.profile:
         # only the kq_quantize launches of the largest shape (for ncu captures)
-        w, p, _, slots = rings[dominant]
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
         for k in range(W + K):
-            x, codes, scales = slots[k % R]
-            if k >= W:
-                ev[2 * (k - W)].record(stream)
-            kq.kq_quantize(x, p, codes, scales)
-            if k >= W:
-                ev[2 * (k - W) + 1].record(stream)
+            launch(dominant, k, "kq")
         torch.cuda.synchronize(device)
-        us = [ev[2 * i].elapsed_time(ev[2 * i + 1]) * 1e3 for i in range(K)]
+        us = timed_burst(dominant, "kq", K, 0) * 1e3
+        w = ws[dominant]
         if rank == 0:
-            print(json.dumps({"profile": f"kq_quantize {w.M}x{w.d}", "launches": W + K,
-                              "us_per_launch": round(sum(us) / K, 2),
-                              "gbs": round(algorithmic_bytes(w.M, w.d) / (sum(us) / K * 1e-6) / 1e9, 1),
+            print(json.dumps({"profile": f"kq_quantize {w.M}x{w.d}", "launches": W + 2 * K,
+                              "us_per_launch": round(us, 2),
+                              "gbs": round(algorithmic_bytes(w.M, w.d) / (us * 1e-6) / 1e9, 1),
                               "device_status": kq.kq_device_status(device)}), flush=True)
         return 0
     sampler = ClockSampler(device.index if device.index is not None else 0).start()
-    ms_kq, launch_kq, t0, t1 = timed("kq", K, W, per_launch=True)
+    ms_kq, t0, t1 = timed_steps("kq", K, W)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
-    ms_sq, launch_sq, _, _ = timed("sq", K, W, per_launch=True)
+    ms_sq, _, _ = timed_steps("sq", K, W)
+    launch_kq = [timed_burst(i, "kq", K, W) for i in range(len(rings))]
+    launch_sq = [timed_burst(i, "sq", K, W) for i in range(len(rings))]
+    launch_tc = timed_burst(dominant, "tc", K, W)
 
     # end to end through the public API: pinned host input -> device -> quantize -> host
     host_out = [(torch.empty((w.M, w.d // 2), dtype=torch.uint8).pin_memory(),
@@ -346,7 +355,7 @@ def run_kroquant(args) -> int:
 
     def e2e_step(k):
         for i, (w, p, _, slots) in enumerate(rings):
-            x, codes, scales = slots[k % R]
+            x, codes, scales = slots[k % len(slots)]
             x.copy_(host_pinned[i], non_blocking=True)
             kq.kq_quantize(x, p, codes, scales)
             host_out[i][0].copy_(codes, non_blocking=True)
@@ -412,9 +421,11 @@ def run_kroquant(args) -> int:
                             "one kq_quantize launch per shape per step",
                 "M_per_rank": ws[0].M,
                 "d": [w.d for w in ws],
-                "l2": f"inputs larger than L2: ring of {R} distinct input/output sets "
-                      f"({R * step_bytes(ws) / 1e6:.0f} MB > {RING_FACTOR_L2:.0f} x L2 "
-                      f"{l2 / 2 ** 20:.0f} MiB)",
+                "l2": "inputs larger than L2: each shape cycles through its own ring of "
+                      + ", ".join(f"{r} (d={w.d}, {r * algorithmic_bytes(w.M, w.d) / 1e6:.0f} MB)"
+                                  for r, w in zip(Rs, ws))
+                      + f" distinct input/output sets, each ring > {RING_FACTOR_L2:.0f} x L2 "
+                        f"({l2 / 2 ** 20:.0f} MiB)",
                 "parallelism": f"replicas x{world} (token rows per rank, no collective)",
             },
             "gpu_launches": K * len(ws),
@@ -427,6 +438,7 @@ def run_kroquant(args) -> int:
                 "frac": round(achieved / peak, 4),
                 "traffic": traffic,
                 "algorithmic_bytes_per_launch": dom_bytes,
+                "timing": "mean of K back-to-back launches of this shape between two CUDA events",
                 "peak_source": peak_src,
                 "traffic_source": traffic_src,
             },
@@ -437,6 +449,12 @@ def run_kroquant(args) -> int:
                 "context": PAGES_CONTEXT,
             },
             "per_shape": per_shape,
+            "tensor_core_variant": {
+                "kernel": f"kq_quantize_tc {wd.M}x{wd.d} (tcgen05 MMAs of the dense 32x32 blocks)",
+                "us": round(launch_tc * 1e3, 2),
+                "gbs": round(dom_bytes / (launch_tc * 1e-3) / 1e9, 1),
+                "frac_of_peak": round(dom_bytes / (launch_tc * 1e-3) / 1e9 / peak, 4),
+            },
             "e2e": {
                 "value": round(e2e_value, 2),
                 "unit": UNIT,

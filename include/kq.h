@@ -89,6 +89,20 @@ int kq_quantize(const void* x, int x_dtype, int64_t M, int64_t d,
                 void* stream);
 
 /*
+ * kq_quantize_tc -- the same operation as kq_quantize, computed the way the
+ * method's own kernel does it ("small tensor-core GEMMs", Abstract): each
+ * 32 x 32 block transform runs on the tcgen05 tensor cores (T_j expanded in
+ * fp32 and split into three bf16 terms, fp32 accumulation in tensor memory)
+ * and the SIMT warps only encode.  bf16 input only (KQ_ERR_DTYPE otherwise);
+ * other arguments, layouts, limits and tolerances as kq_quantize.  On B200 at
+ * DiT shapes it is slower than kq_quantize's packed-FP32 shear butterfly; it
+ * is kept for that comparison.
+ */
+int kq_quantize_tc(const void* x, int x_dtype, int64_t M, int64_t d,
+                   const float* params, uint8_t* codes, uint8_t* scales,
+                   void* stream);
+
+/*
  * kq_transform -- the transform stage alone: y = blockdiag(T_j) x in fp32.
  * Same arguments and limits as kq_quantize; y [M][d] fp32, 16-byte aligned.
  * It runs the same transform code as kq_quantize, so kq_quantize's codes are

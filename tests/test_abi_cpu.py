@@ -28,7 +28,7 @@ def header_functions():
 
 def test_header_declares_the_abi():
     names = header_functions()
-    for want in ("kq_quantize", "kq_transform", "sq_quantize", "kq_expand_params",
+    for want in ("kq_quantize", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
                  "kq_fold_weights", "kq_dequant", "kq_status_string", "kq_device_status"):
         assert want in names
 
@@ -81,6 +81,14 @@ def test_quantize_argument_checks(lib):
     assert q(None, 0, 0, 64, None, None, None, None) == 0          # ... pointers unused
     assert q(None, 0, 0, 48, None, None, None, None) == 1          # shape still checked
     assert b"kq_quantize" in lib.kq_last_error()
+
+
+def test_tensor_core_variant_checks(lib):
+    t = lib.kq_quantize_tc
+    assert t(A16, 1, 4, 64, A16b, A16c, A16d, None) == 3          # fp32 input refused
+    assert t(A16, 0, 4, 48, A16b, A16c, A16d, None) == 1
+    assert t(A16 + 8, 0, 4, 64, A16b, A16c, A16d, None) == 2
+    assert t(None, 0, 0, 64, None, None, None, None) == 0          # M == 0
 
 
 def test_other_argument_checks(lib):

@@ -304,3 +304,41 @@ def test_empty_input(kq):
     p = torch.zeros((2, 15), device="cuda")
     codes, scales = kq.kq_quantize(x, p)
     assert codes.shape == (0, 32) and scales.shape == (0, 2)
+
+
+# ---------------------------------------------------------------------------
+# the tensor-core formulation (kq_quantize_tc): same contract
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,d", [(1, 32), (129, 96), (200, 1152), (1031, 224), (333, 5600)])
+def test_tensor_core_small(kq, M, d):
+    w = synthetic.Workload("tcs", M, d, "bf16", "normal", 0.05, None, 40.0, 2.0, 19)
+    raw = synthetic.make_activations(w)
+    p, pd = params_dev(w.nb, 6)
+    codes, cw = padded_u8((M, d // 2))
+    scales, sw = padded_u8((M, d // 32))
+    kq.kq_quantize_tc(to_device(raw, "bf16"), pd, codes, scales)
+    torch.cuda.synchronize()
+    assert guards_intact(cw, M * d // 2) and guards_intact(sw, M * d // 32)
+    y_ref, tol = reference(f64(raw, "bf16"), params=p)
+    check(compare_codes(codes.cpu().numpy(), scales.cpu().numpy(), y_ref, tol), f"tc {M}x{d}")
+
+
+@pytest.mark.parametrize("w", synthetic.workloads(["pixart", "sana", "flux"]), ids=lambda w: w.key)
+def test_tensor_core_workloads(kq, w):
+    xd = device_activations(w)
+    p, pd = params_dev(w.nb, w.seed)
+    codes, scales = kq.kq_quantize_tc(xd, pd)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.M, 384, w.seed)
+    y_ref, tol = reference(f64(synthetic.make_activations(w, rows), w.dtype), params=p)
+    check(compare_codes(codes[rows].cpu().numpy(), scales[rows].cpu().numpy(), y_ref, tol), f"tc {w.key}")
+
+
+def test_tensor_core_exact_identity(kq):
+    w = synthetic.Workload("tci", 300, 1024, "bf16", "normal", 0.02, None, 50.0, 1.0, 26)
+    raw = synthetic.make_activations(w)
+    p = synthetic.identity_params(w.nb)
+    codes, scales = kq.kq_quantize_tc(to_device(raw, "bf16"), torch.from_numpy(p).cuda())
+    c_ref, s_ref = o.quantize_mxfp4(f64(raw, "bf16"))
+    assert np.array_equal(scales.cpu().numpy(), s_ref)
+    assert np.array_equal(codes.cpu().numpy(), c_ref)

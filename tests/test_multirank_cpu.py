@@ -65,5 +65,5 @@ def test_rank_plan_and_bytes():
     assert bench.algorithmic_bytes(4608, 12288) == 4608 * 12288 * 2.53125 + 384 * 60
     # the ring of input/output sets exceeds four times L2
     l2 = 126 * 2 ** 20
-    R = bench.ring_depth(ws, l2)
-    assert R * sum(w.M * w.d * 2.53125 for w in ws) >= 4 * l2
+    for w in ws:
+        assert bench.ring_depth(w, l2) * w.M * w.d * 2.53125 >= 4 * l2

@@ -19,7 +19,7 @@ import torch
 from .build import LIB_PATH
 
 __all__ = [
-    "abi", "kq_quantize", "kq_transform", "sq_quantize", "kq_expand_params",
+    "abi", "kq_quantize", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
     "kq_fold_weights", "kq_dequant", "kq_device_status", "KroQuantError",
     "KQ_DTYPE_BF16", "KQ_DTYPE_F32", "KQ_MAX_D", "EXPORTED_FUNCTIONS",
 ]
@@ -36,6 +36,7 @@ _int = ctypes.c_int
 # name -> (restype, argtypes), mirroring include/kq.h
 _SIGNATURES = {
     "kq_quantize": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "kq_quantize_tc": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_transform": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
     "sq_quantize": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_expand_params": (_int, [_c_void_p, _i64, _c_void_p, _c_void_p]),
@@ -130,6 +131,21 @@ def kq_quantize(x, params, codes=None, scales=None):
     with torch.cuda.device(x.device):
         _check("kq_quantize", abi().kq_quantize(
             x.data_ptr(), _x_dtype(x), M, d, params.data_ptr(), codes.data_ptr(),
+            scales.data_ptr(), _stream(x)))
+    return codes, scales
+
+
+def kq_quantize_tc(x, params, codes=None, scales=None):
+    """Same result contract as kq_quantize, computed on the tensor cores
+    (bf16 input only); kept for comparison with the SIMT path."""
+    _need_cuda("x", x, (torch.bfloat16,), 2)
+    _need_cuda("params", params, (torch.float32,))
+    M, d = x.shape
+    codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
+    scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
+    with torch.cuda.device(x.device):
+        _check("kq_quantize_tc", abi().kq_quantize_tc(
+            x.data_ptr(), KQ_DTYPE_BF16, M, d, params.data_ptr(), codes.data_ptr(),
             scales.data_ptr(), _stream(x)))
     return codes, scales
 

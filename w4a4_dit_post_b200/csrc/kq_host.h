@@ -27,6 +27,10 @@ int sm_count(int* out);
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Device address of the per-device status word (defined in kq_stream.cu),
+// for kernels compiled in other translation units; cached per device.
+int device_status_address(unsigned int** out);
+
 // Common checks of (M, d): M >= 0, d > 0, d % 32 == 0, d <= max_d,
 // M * d / 32 < 2^31.
 int check_shape(int64_t M, int64_t d, int64_t max_d, const char* fn);

@@ -253,6 +253,11 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   const int j0 = col_group * C;                 // first block column of the group
   const uint32_t tile_tx = (uint32_t)(R * C * InLayout<kInBytes>::kBlockBytes);
 
+  // Programmatic dependent launch: let the next kernel in the stream begin
+  // launching now, and touch no global memory before the previous kernel in
+  // the stream has completed (griddepcontrol.wait returns at once when this
+  // launch has no programmatic predecessor).
+  pdl_launch_dependents();
   if (tid == 0) {
     tma_prefetch_desc(&tmap);
 #pragma unroll
@@ -260,6 +265,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
     *abort_flag = 0;
     mbar_init_fence();
   }
+  pdl_wait_predecessor();
   __syncthreads();
   if (tid == 0) {
 #pragma unroll
@@ -469,7 +475,19 @@ int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_
   if (per_group < 1) per_group = 1;
   if (per_group > geo.n_row_tiles) per_group = geo.n_row_tiles;
   const int64_t grid = per_group * geo.NC;
-  kern<<<(unsigned)grid, kThreads, smem, stream>>>(tm, coef, geo, codes, scales, y);
+  // launched with programmatic stream serialization (see the kernel's prologue)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, tm, coef, geo, codes, scales, y);
+  if (err != cudaSuccess) return cuda_fail(err, "stream_kernel launch");
   return check_launch("stream_kernel launch");
 }
 
@@ -496,6 +514,28 @@ int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef
 }
 
 }  // namespace
+}  // namespace kq
+
+namespace kq {
+
+int device_status_address(unsigned int** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
+  static std::mutex mu;
+  static unsigned int* addr[64] = {nullptr};
+  if (dev < 0 || dev >= 64) return fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_devstat);
+    if (err != cudaSuccess) return cuda_fail(err, "cudaGetSymbolAddress(status word)");
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  *out = addr[dev];
+  return KQ_OK;
+}
+
 }  // namespace kq
 
 extern "C" {
