@@ -328,14 +328,16 @@ def run_kroquant(args) -> int:
 
     K, W = args.steps, args.warmup
     if args.profile:
-        # only the kq_quantize launches of the largest shape (for ncu captures)
+        # only the launches of one kernel on the largest shape (for ncu captures)
+        fn = "tc" if args.profile == "tc" else "kq"
         for k in range(W + K):
-            launch(dominant, k, "kq")
+            launch(dominant, k, fn)
         torch.cuda.synchronize(device)
-        us = timed_burst(dominant, "kq", K, 0) * 1e3
+        us = timed_burst(dominant, fn, K, 0) * 1e3
         w = ws[dominant]
+        name = "kq_quantize_tc" if fn == "tc" else "kq_quantize"
         if rank == 0:
-            print(json.dumps({"profile": f"kq_quantize {w.M}x{w.d}", "launches": W + 2 * K,
+            print(json.dumps({"profile": f"{name} {w.M}x{w.d}", "launches": W + 2 * K,
                               "us_per_launch": round(us, 2),
                               "gbs": round(algorithmic_bytes(w.M, w.d) / (us * 1e-6) / 1e9, 1),
                               "device_status": kq.kq_device_status(device)}), flush=True)
@@ -559,8 +561,9 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["kroquant", "reference"], default="kroquant")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", action="store_true",
-                    help="run only the kq_quantize launches of the largest shape (ncu captures)")
+    ap.add_argument("--profile", nargs="?", const="kq", choices=["kq", "tc"], default=None,
+                    help="run only the kq_quantize (or kq_quantize_tc) launches of the largest "
+                         "shape, for ncu captures")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     _, world, _ = dist_env()

@@ -160,6 +160,17 @@ int kq_dequant(const uint8_t* codes, const uint8_t* scales, int64_t M, int64_t d
  */
 int kq_device_status(uint32_t* flags, int clear);
 
+/*
+ * kq_selftest_bounded_wait -- failure-detection self-test.  Enqueues a kernel
+ * whose one thread waits, through the same bounded wait the streaming
+ * kernels use, on a shared-memory barrier that nothing arrives on.  After
+ * limit_us microseconds (1 .. 1e6) the wait gives up, the kernel sets
+ * KQ_DEVSTAT_WAIT_TIMEOUT in the device status word and returns; nothing
+ * faults and the context stays usable.  Read and clear the bit with
+ * kq_device_status().  Not part of the method (no page describes it).
+ */
+int kq_selftest_bounded_wait(uint32_t limit_us, void* stream);
+
 /* Static text for a status code (never NULL). */
 const char* kq_status_string(int status);
 

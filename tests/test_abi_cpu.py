@@ -105,6 +105,8 @@ def test_other_argument_checks(lib):
     assert lib.kq_dequant(A16, A16b, 4, 64, A16c + 4, None) == 2
     assert lib.kq_dequant(A16, A16b, 0, 64, A16c, None) == 0
     assert lib.kq_device_status(None, 0) == 1
+    assert lib.kq_selftest_bounded_wait(0, None) == 1
+    assert lib.kq_selftest_bounded_wait(2000000, None) == 1
 
 
 def test_binding_refuses_host_tensors(lib):

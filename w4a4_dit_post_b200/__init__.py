@@ -20,7 +20,8 @@ from .build import LIB_PATH
 
 __all__ = [
     "abi", "kq_quantize", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
-    "kq_fold_weights", "kq_dequant", "kq_device_status", "KroQuantError",
+    "kq_fold_weights", "kq_dequant", "kq_device_status", "kq_selftest_bounded_wait",
+    "KroQuantError",
     "KQ_DTYPE_BF16", "KQ_DTYPE_F32", "KQ_MAX_D", "EXPORTED_FUNCTIONS",
 ]
 
@@ -43,6 +44,7 @@ _SIGNATURES = {
     "kq_fold_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
     "kq_dequant": (_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "kq_device_status": (_int, [ctypes.POINTER(ctypes.c_uint32), _int]),
+    "kq_selftest_bounded_wait": (_int, [ctypes.c_uint32, _c_void_p]),
     "kq_status_string": (ctypes.c_char_p, [_int]),
     "kq_last_error": (ctypes.c_char_p, []),
     "kq_version": (_int, []),
@@ -221,3 +223,11 @@ def kq_device_status(device=None, clear: bool = False) -> int:
     with torch.cuda.device(dev):
         _check("kq_device_status", abi().kq_device_status(ctypes.byref(flags), int(bool(clear))))
     return flags.value
+
+
+def kq_selftest_bounded_wait(limit_us: int, device=None) -> None:
+    """Enqueue the bounded-wait self-test on the current stream of `device`."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check("kq_selftest_bounded_wait", abi().kq_selftest_bounded_wait(
+            int(limit_us), torch.cuda.current_stream(dev).cuda_stream))

@@ -391,6 +391,18 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   }
 }
 
+// Failure-detection self-test: one thread waits on a barrier that nothing
+// arrives on, through the same bounded wait the streaming kernels use.  The
+// wait runs out after limit_ns, sets the status bit and the kernel returns.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(smem_addr(&bar), 1);
+  mbar_init_fence();
+  if (!mbar_wait_bounded(smem_addr(&bar), 0u, limit_ns))
+    atomicOr(&g_devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -556,6 +568,14 @@ int sq_quantize(const void* x, int x_dtype, int64_t M, int64_t d, const float* i
                 uint8_t* codes, uint8_t* scales, void* stream) {
   return kq::dispatch<kq::Op::kSqQuant>(x, x_dtype, M, d, inv_s, codes, scales, nullptr, stream,
                                         "sq_quantize");
+}
+
+int kq_selftest_bounded_wait(uint32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_selftest_bounded_wait: limit_us = %u not in [1, 1e6]",
+                    limit_us);
+  kq::selftest_wait_kernel<<<1, 32, 0, kq::as_stream(stream)>>>((uint64_t)limit_us * 1000ull);
+  return kq::check_launch("selftest_wait_kernel launch");
 }
 
 int kq_device_status(uint32_t* flags, int clear) {

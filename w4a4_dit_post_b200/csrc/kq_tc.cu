@@ -141,6 +141,7 @@ struct Layout {
   int table_off;     // after the stages; C * 3 * 2048 bytes
   int out_off;       // two code staging buffers of 128 x C*16 bytes (1024-aligned)
   int out_bytes;
+  int sc_off;        // scale staging, 128 x C bytes
   int bar_off;       // barriers and flags
   int total;
 };
@@ -151,7 +152,8 @@ __host__ __device__ inline Layout layout_for(int C) {
   L.table_off = kStages * L.stage_bytes;
   L.out_off = L.table_off + C * 3 * 2048;
   L.out_bytes = ((kRows * C * 16) + 1023) & ~1023;
-  L.bar_off = L.out_off + 2 * L.out_bytes;
+  L.sc_off = L.out_off + 2 * L.out_bytes;       // scale bytes of one tile: 128 x C
+  L.bar_off = L.sc_off + ((kRows * C + 127) & ~127);
   L.total = L.bar_off + 256;
   return L;
 }
@@ -349,6 +351,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUte
       const int rt = rt_first + it * row_step;
       const int row = rt * kRows + r_local;
       uint8_t* stage_out = smem + L.out_off + a * L.out_bytes;
+      uint8_t* stage_sc = smem + L.sc_off;
       const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)a * acc_cols;
       auto emit = [&](int jj, const float2 (&v)[16]) {
         if constexpr (kTransformOnly) {
@@ -362,7 +365,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUte
           uint4 packed;
           const uint32_t byte = mxfp4_encode32(v, packed);
           *reinterpret_cast<uint4*>(stage_out + out_offset(C, r_local, jj)) = packed;
-          if (row < geo.M) scales[(size_t)row * nb + j0 + jj] = (uint8_t)byte;
+          stage_sc[r_local * C + jj] = (uint8_t)byte;
         }
       };
       int jj = jj_lo;
@@ -387,6 +390,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUte
         if (tid == 0) {
           tma_store_2d(&omap, j0 * 16, rt * kRows, smem_addr(stage_out));
           bulk_commit();
+        }
+        // scale bytes: consecutive threads write consecutive bytes of a row
+        for (int i = tid; i < kRows * C; i += kEpiWarps * 32) {
+          const int r = i / C, c = i - r * C;
+          const int grow = rt * kRows + r;
+          if (grow < geo.M) scales[(size_t)grow * nb + j0 + c] = stage_sc[i];
         }
       }
     }
