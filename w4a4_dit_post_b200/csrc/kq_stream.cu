@@ -257,6 +257,12 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   // launching now, and touch no global memory before the previous kernel in
   // the stream has completed (griddepcontrol.wait returns at once when this
   // launch has no programmatic predecessor).
+  //
+  // Before that wait the CTA only asks for its first tiles and its
+  // coefficients to be brought into L2.  A prefetch changes no memory and L2
+  // is where every write of the previous kernel lands, so the loads after the
+  // wait still see that kernel's results; they just find them on chip.  This
+  // overlaps the start of this launch with the tail of the previous one.
   pdl_launch_dependents();
   if (tid == 0) {
     tma_prefetch_desc(&tmap);
@@ -264,6 +270,18 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
     for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
     *abort_flag = 0;
     mbar_init_fence();
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+      const int rt = rt_first + s * row_step;
+      if (rt < geo.n_row_tiles) tma_prefetch_l2_3d(&tmap, 0, j0, rt * R);
+    }
+  }
+  {
+    constexpr int kCoefPerBlock = (kOp == Op::kSqQuant) ? 32 : 15;
+    const char* cbase = reinterpret_cast<const char*>(coef_src + kCoefPerBlock * j0);
+    const int cbytes = C * kCoefPerBlock * 4;
+    const int first = tid * 128 - (int)(reinterpret_cast<uintptr_t>(cbase) & 127);
+    if (tid < 32 && first < cbytes) prefetch_l2(cbase + (first > 0 ? first : 0));
   }
   pdl_wait_predecessor();
   __syncthreads();

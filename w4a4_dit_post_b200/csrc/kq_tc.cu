@@ -2,34 +2,35 @@
 //
 // The per-block transform y = T_j x (a 32 x 32 contraction per token and
 // block column) runs on the 5th-generation tensor cores as small GEMMs --
-// the "small tensor-core GEMMs" of the method -- and the SIMT warps only
-// encode.  Exactness: x is bf16 (exact operand); T_j is expanded in fp32 and
-// split into three bf16 terms T = T_hi + T_mid + T_lo (residual below 2^-27
-// |T|), each multiplied exactly and accumulated in fp32 in tensor memory.
+// the "small tensor-core GEMMs" option of the method -- and the SIMT warps
+// only encode.  Exactness: x is bf16 (an exact operand); T_j is expanded in
+// fp32 and split into three bf16 terms T = T_hi + T_mid + T_lo (residual
+// below 2^-24 |T|), each multiplied exactly and accumulated in fp32 in
+// tensor memory.
 //
-// Work split.  Block columns are cut into NC groups of C <= 8 (C = the
-// largest divisor of nb not above 8); a CTA owns one group for its life
-// (grid = a multiple of NC, one CTA per SM) and walks row tiles of 128 rows.
-// A tile arrives by one 3-D TMA load of the view [nb][M][32] (box 32 x 128 x
-// C): each block column lands as 128 contiguous 64-byte rows with the 64-byte
-// swizzle, which is the canonical K-major SW64 operand layout of tcgen05.mma.
-// The CTA's T splits (C x 3 x 2 KiB, same layout) are built once in shared
-// memory from the LU parameters.
+// Work split.  Block columns are cut into NC groups of C <= 4 (C = the
+// largest divisor of nb not above 4).  A work unit is one group x one tile
+// of 128 token rows; units are numbered group-major and every CTA (one per
+// SM) takes one contiguous, balanced range of them, so that it meets at most
+// three groups and keeps their T splits resident in shared memory.  A unit
+// arrives by one 3-D TMA load of the view [nb][M][32] (box 32 x 128 x C):
+// each block column lands as 128 contiguous 64-byte rows with the 64-byte
+// swizzle, which is the canonical K-major SW64 operand layout of
+// tcgen05.mma.
 //
-// Roles (576 threads):
-//   warp 16, lane 0: TMA producer (two shared-memory stages);
-//   warp 17        : allocates tensor memory; lane 0 issues the MMAs:
-//                    per block column jj: 3 splits x 2 K-steps of
-//                    M=128 x N=32 x K=16 into accumulator columns jj*32..;
-//                    two accumulators of C*32 columns (double buffer);
-//   warps 0..15    : epilogue.  Warp w reads TMEM lanes 32*(w%4).. (its token
-//                    rows) for the block columns of quarter (w/4) of the group
-//                    with tcgen05.ld 32x32b.x32 (one token's block per
-//                    thread, up to two loads in flight), encodes into a
-//                    swizzled shared tile, and one thread stores the tile
-//                    of codes with a TMA tensor store.
+// Roles (320 threads):
+//   warp 8, lane 0: TMA producer (S shared-memory stages, S * C * 8 KiB <= 128 KiB);
+//   warp 9        : allocates tensor memory; lane 0 issues the MMAs:
+//                   per block column jj: 3 splits x 2 K-steps of
+//                   M=128 x N=32 x K=16 into accumulator columns jj*32..;
+//                   four accumulators of 128 columns;
+//   warps 0..7    : epilogue.  Warp w reads TMEM lanes 32*(w%4).. (its token
+//                   rows) for half (w/4) of the unit's block columns with
+//                   tcgen05.ld 32x32b.x32 (one token's block per thread),
+//                   hands the accumulator back, and writes the MXFP4 codes
+//                   (16 bytes) and scale of each block straight to memory.
 // Every mbarrier wait is bounded; a wait that runs out sets the device status
-// word and the CTA drains and exits.
+// word and the CTA drains its copies and MMAs and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -46,14 +47,18 @@
 namespace kq {
 namespace tc {
 
-constexpr int kEpiWarps = 16;
+constexpr int kEpiWarps = 8;
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps;
 constexpr int kMmaWarp = kEpiWarps + 1;
-constexpr int kRows = 128;        // MMA M = token rows per tile
-constexpr int kMaxC = 8;
-constexpr int kStages = 2;
-constexpr int kTmemCols = 512;    // two accumulators of up to 8 x 32 columns
+constexpr int kRows = 128;         // MMA M = token rows per unit
+constexpr int kMaxC = 4;
+constexpr int kMaxGroups = 3;      // table slots: column groups one CTA may meet
+constexpr int kAcc = 4;            // accumulator buffers
+constexpr int kAccCols = 128;      // TMEM columns per accumulator (C * 32 used)
+constexpr int kTmemCols = kAcc * kAccCols;
+constexpr int kStageBudget = 128 * 1024;
+constexpr int kMaxStages = 16;
 
 // UMMA instruction descriptor: D fp32, A and B bf16, both K-major, N = 32, M = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((32u >> 3) << 17) |
@@ -135,105 +140,76 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t t0, uint32_t t1, float2 (&v
   }
 }
 
+
 // Shared-memory layout (offsets from the 1024-aligned base).
 struct Layout {
+  int stages;        // S
   int stage_bytes;   // C * 128 * 64
-  int table_off;     // after the stages; C * 3 * 2048 bytes
-  int out_off;       // two code staging buffers of 128 x C*16 bytes (1024-aligned)
-  int out_bytes;
-  int sc_off;        // scale staging, 128 x C bytes
-  int bar_off;       // barriers and flags
+  int table_off;     // kMaxGroups * C * 3 * 2048 bytes of T splits
+  int fac_off;       // kMaxGroups * C * 5 float4 LU factors (set-up only)
+  int bar_off;       // 2 S + 2 kAcc barriers, abort flag, TMEM address
   int total;
 };
 
 __host__ __device__ inline Layout layout_for(int C) {
   Layout L;
   L.stage_bytes = C * kRows * 64;
-  L.table_off = kStages * L.stage_bytes;
-  L.out_off = L.table_off + C * 3 * 2048;
-  L.out_bytes = ((kRows * C * 16) + 1023) & ~1023;
-  L.sc_off = L.out_off + 2 * L.out_bytes;       // scale bytes of one tile: 128 x C
-  L.bar_off = L.sc_off + ((kRows * C + 127) & ~127);
-  L.total = L.bar_off + 256;
+  L.stages = kStageBudget / L.stage_bytes;
+  if (L.stages > kMaxStages) L.stages = kMaxStages;
+  L.table_off = L.stages * L.stage_bytes;
+  L.fac_off = L.table_off + kMaxGroups * C * 3 * 2048;
+  L.bar_off = L.fac_off + 1024;
+  L.total = L.bar_off + 512;
   return L;
 }
 
-// Staging position of (token row r, block jj) in a code tile of C*16-byte rows.
-// With C == 8 the rows are 128 bytes and the 128-byte swizzle (chunk ^ r % 8)
-// keeps the per-row 16-byte writes conflict-free; the TMA store map matches.
-__device__ __forceinline__ int out_offset(int C, int r, int jj) {
-  return C == 8 ? r * 128 + ((jj ^ (r & 7)) << 4) : (r * C + jj) * 16;
-}
-
-__device__ __forceinline__ void tma_store_2d(const void* tmap, int c0, int c1, uint32_t src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
-               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(src)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Barrier 1 among the epilogue warps only (the producer and MMA warps never
-// take part).  epi_any also ORs a flag across them, so every epilogue warp
-// takes the same branch after it (no warp can leave another waiting).
-__device__ __forceinline__ void epi_barrier() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");
-}
-__device__ __forceinline__ bool epi_any(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(kEpiWarps * 32)
-      : "memory");
-  return r != 0;
-}
-
-template <bool kTransformOnly>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap omap,
-          const float* __restrict__ params,
+tc_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ params,
           const TcGeometry geo, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-          float* __restrict__ y_out, unsigned int* devstat) {
+          unsigned int* devstat) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int C = geo.C;
   const Layout L = layout_for(C);
+  const int S = L.stages;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  // bars: full[2], empty[2], acc_full[2], acc_empty[2]
-  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[2]);
-  const uint32_t accf0 = smem_addr(&bars[4]), acce0 = smem_addr(&bars[6]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bar_off + 64);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.bar_off + 128);
+  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[S]);
+  const uint32_t accf0 = smem_addr(&bars[2 * S]), acce0 = smem_addr(&bars[2 * S + kAcc]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bar_off + 384);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.bar_off + 448);
   const uint32_t table = smem_addr(smem + L.table_off);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int col_group = blockIdx.x % geo.NC;
-  const int row_step = gridDim.x / geo.NC;
-  const int rt_first = blockIdx.x / geo.NC;
-  const int j0 = col_group * C;
-  const int n_items = rt_first < geo.n_row_tiles
-                          ? (geo.n_row_tiles - rt_first + row_step - 1) / row_step
-                          : 0;
+  const int n_rt = geo.n_row_tiles;
+  const int64_t U = (int64_t)geo.NC * n_rt;
+  const int64_t u_begin = (int64_t)blockIdx.x * U / gridDim.x;
+  const int64_t u_end = (int64_t)(blockIdx.x + 1) * U / gridDim.x;
+  const int n_items = (int)(u_end - u_begin);
+  const int g_first = (int)(u_begin / n_rt);
+  const int n_groups = n_items > 0 ? (int)((u_end - 1) / n_rt) - g_first + 1 : 0;
 
   pdl_launch_dependents();
   if (tid == 0) {
     tma_prefetch_desc(&tmap);
-    if (!kTransformOnly) tma_prefetch_desc(&omap);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < S; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < kAcc; ++i) {
       mbar_init(accf0 + 8 * i, 1);
       mbar_init(acce0 + 8 * i, kEpiWarps);
     }
     *abort_flag = 0;
     mbar_init_fence();
+    // L2 prefetch of the first units before the wait on the previous kernel
+    // (a hint that changes no memory; the loads after the wait see that
+    // kernel's writes, which land in L2)
+    for (int it = 0; it < n_items && it < S; ++it) {
+      const int64_t u = u_begin + it;
+      const int g = (int)(u / n_rt), rt = (int)(u - (int64_t)g * n_rt);
+      tma_prefetch_l2_3d(&tmap, 0, rt * kRows, g * C);
+    }
   }
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -243,37 +219,68 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUte
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   pdl_wait_predecessor();
+  __syncthreads();
 
-  // T splits of the C block columns: [jj][part][n = output row][k], bf16,
-  // 64-byte rows with the 64-byte swizzle (chunk ^= (n >> 1) & 3).  The five
-  // factors of each column are computed once (C * 5 threads), then each
-  // thread forms entries T[n][k] = prod_m A_m[bit][bit] and splits them.
-  float4* fac = reinterpret_cast<float4*>(smem + L.out_off);   // staging area, free until the epilogue
-  for (int i = tid; i < C * 5; i += kThreads) {
-    const int jj = i / 5, m = i - 5 * jj;
-    const float* p = params + 15 * (j0 + jj) + 3 * m;
+  // The first S loads go out before the tables are built.
+  const uint32_t tx = (uint32_t)L.stage_bytes;
+  auto issue = [&](int it) {
+    const int64_t u = u_begin + it;
+    const int g = (int)(u / n_rt), rt = (int)(u - (int64_t)g * n_rt);
+    const int s = it % S;
+    mbar_arrive_expect_tx(full0 + 8 * s, tx);
+    tma_load_3d(smem_addr(smem + s * L.stage_bytes), &tmap, 0, rt * kRows, g * C, full0 + 8 * s);
+  };
+  if (warp == kProducerWarp && lane == 0)
+    for (int it = 0; it < n_items && it < S; ++it) issue(it);
+
+  // T splits of the groups this CTA meets: [slot][jj][part][n = output row][k],
+  // bf16, 64-byte rows with the 64-byte swizzle (16-byte chunk ^= (n >> 1) & 3).
+  // First the five LU factors of every block column, then one thread per
+  // output row n expands T[n][.] = prod_m A_m[bit(n)][bit(.)] by Kronecker
+  // doubling (factor 0 on the most significant index bit) and splits it.
+  float4* fac = reinterpret_cast<float4*>(smem + L.fac_off);
+  for (int i = tid; i < n_groups * C * 5; i += kThreads) {
+    const int cj = i / 5, m = i - 5 * cj;   // cj = slot * C + jj
+    const float* p = params + 15 * ((int64_t)g_first * C + cj) + 3 * m;
     fac[i] = lu_factor(p[0], p[1], p[2]);
   }
   __syncthreads();
-  for (int i = tid; i < C * 1024; i += kThreads) {
-    const int jj = i >> 10, n = (i >> 5) & 31, k = i & 31;
-    float t = 1.0f;
+  for (int ri = tid; ri < n_groups * C * 32; ri += kThreads) {
+    const int cj = ri >> 5, n = ri & 31;
+    float t[32];
+    t[0] = 1.0f;
 #pragma unroll
     for (int m = 0; m < 5; ++m) {
-      const float4 A = fac[jj * 5 + m];
-      const int bn = (n >> (4 - m)) & 1, bk = (k >> (4 - m)) & 1;
-      t = __fmul_rn(t, bn ? (bk ? A.w : A.z) : (bk ? A.y : A.x));
+      const float4 A = fac[cj * 5 + m];
+      const bool hi_row = (n >> (4 - m)) & 1;
+      const float a0 = hi_row ? A.z : A.x, a1 = hi_row ? A.w : A.y;
+#pragma unroll
+      for (int q = (1 << m) - 1; q >= 0; --q) {
+        t[2 * q + 1] = __fmul_rn(t[q], a1);
+        t[2 * q] = __fmul_rn(t[q], a0);
+      }
     }
-    const __nv_bfloat16 hi = __float2bfloat16_rn(t);
-    const float r1 = t - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-    const int off = n * 64 + ((((k >> 3) ^ ((n >> 1) & 3))) << 4) + (k & 7) * 2;
-    __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(smem + L.table_off + jj * 3 * 2048);
-    base[(0 * 2048 + off) / 2] = hi;
-    base[(1 * 2048 + off) / 2] = mid;
-    base[(2 * 2048 + off) / 2] = lo;
+    uint8_t* rowp = smem + L.table_off + cj * 3 * 2048 + n * 64;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t w[3][4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = t[8 * ch + 2 * e], x1 = t[8 * ch + 2 * e + 1];
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+        const float r0 = x0 - __low2float(h), r1 = x1 - __high2float(h);
+        const __nv_bfloat162 mid = __floats2bfloat162_rn(r0, r1);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(r0 - __low2float(mid), r1 - __high2float(mid));
+        w[0][e] = *reinterpret_cast<const uint32_t*>(&h);
+        w[1][e] = *reinterpret_cast<const uint32_t*>(&mid);
+        w[2][e] = *reinterpret_cast<const uint32_t*>(&lo);
+      }
+      const int off = ((ch ^ ((n >> 1) & 3))) << 4;
+#pragma unroll
+      for (int part = 0; part < 3; ++part)
+        *reinterpret_cast<uint4*>(rowp + part * 2048 + off) =
+            make_uint4(w[part][0], w[part][1], w[part][2], w[part][3]);
+    }
   }
   // make the generic-proxy table writes visible to the tensor cores
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -281,125 +288,119 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUte
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t acc_cols = (uint32_t)(C * 32);
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      const uint32_t tx = (uint32_t)L.stage_bytes;
-      for (int it = 0; it < n_items; ++it) {
-        const int s = it & 1;
-        if (it >= 2 && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)((it >> 1) - 1) & 1u)) {
+      int issued = n_items < S ? n_items : S;
+      for (int it = S; it < n_items; ++it) {
+        const int s = it % S;
+        if (!mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(it / S - 1) & 1u)) {
           *abort_flag = 1;
           atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
           break;
         }
         if (*abort_flag) break;
-        const int rt = rt_first + it * row_step;
-        mbar_arrive_expect_tx(full0 + 8 * s, tx);
-        tma_load_3d(smem_addr(smem + s * L.stage_bytes), &tmap, 0, rt * kRows, j0, full0 + 8 * s);
+        issue(it);
+        issued = it + 1;
+      }
+      // after an abort, let the copies still in flight land before the
+      // shared memory goes away (on the normal path these return at once)
+      if (*abort_flag) {
+        const int lo = issued > S ? issued - S : 0;
+        for (int it = lo; it < issued; ++it)
+          (void)mbar_wait_bounded(full0 + 8 * (it % S), (uint32_t)(it / S) & 1u);
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
+      int done = 0;
       for (int it = 0; it < n_items; ++it) {
-        const int s = it & 1, a = it & 1;
-        const bool ok_full = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(it >> 1) & 1u);
-        const bool ok_acc = it < 2 || mbar_wait_bounded(acce0 + 8 * a, (uint32_t)((it >> 1) - 1) & 1u);
+        const int s = it % S, a = it % kAcc;
+        const bool ok_full = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(it / S) & 1u);
+        const bool ok_acc =
+            it < kAcc || mbar_wait_bounded(acce0 + 8 * a, (uint32_t)(it / kAcc - 1) & 1u);
         if (!ok_full || !ok_acc || *abort_flag) {
           *abort_flag = 1;
           atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
           break;
         }
         fence_after_sync();
+        const int64_t u = u_begin + it;
+        const int slot = (int)(u / n_rt) - g_first;
         const uint32_t a_base = smem_addr(smem + s * L.stage_bytes);
+        const uint32_t t_base = table + (uint32_t)(slot * C * 3 * 2048);
         for (int jj = 0; jj < C; ++jj) {
-          const uint32_t d = tmem_base + (uint32_t)a * acc_cols + (uint32_t)(jj * 32);
+          const uint32_t d = tmem_base + (uint32_t)(a * kAccCols + jj * 32);
 #pragma unroll
           for (int part = 0; part < 3; ++part) {
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
               const uint64_t adesc = sw64_desc(a_base + jj * (kRows * 64) + ks * 32);
-              const uint64_t bdesc = sw64_desc(table + (jj * 3 + part) * 2048 + ks * 32);
+              const uint64_t bdesc = sw64_desc(t_base + (jj * 3 + part) * 2048 + ks * 32);
               mma_bf16(d, adesc, bdesc, (part | ks) != 0);
             }
           }
         }
         mma_commit(empty0 + 8 * s);   // shared-memory stage free once these MMAs are done
         mma_commit(accf0 + 8 * a);    // accumulator ready for the epilogue
+        done = it + 1;
       }
+      // after an abort, wait (bounded) for the last MMAs before TMEM and the
+      // stages are released; MMAs complete in issue order
+      if (*abort_flag && done > 0)
+        (void)mbar_wait_bounded(accf0 + 8 * ((done - 1) % kAcc), (uint32_t)((done - 1) / kAcc) & 1u);
     }
   } else {
-    // epilogue warps
+    // epilogue warps: no barrier among them, so a warp that stops early
+    // leaves nobody waiting except through bounded mbarrier waits
     const int q = warp & 3;                 // TMEM lane quarter = token rows 32q..32q+31
-    const int slot = warp >> 2;             // which quarter of the group's block columns
-    const int jj_lo = (slot * C) / 4;
-    const int jj_hi = ((slot + 1) * C) / 4;
+    const int h = warp >> 2;                // which half of the unit's block columns
+    const int jj_lo = (h * C) / 2, jj_hi = ((h + 1) * C) / 2;
     const int nb = geo.nb;
-    const int r_local = 32 * q + lane;      // token row inside the tile
     for (int it = 0; it < n_items; ++it) {
-      const int a = it & 1;
-      const bool ok = mbar_wait_bounded(accf0 + 8 * a, (uint32_t)(it >> 1) & 1u);
-      if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
-      // the TMA store that last read this staging buffer (item it - 2) is done
-      if (!kTransformOnly && tid == 0) bulk_wait_read_1();
-      // one decision for all epilogue warps (also the staging-buffer barrier)
-      if (epi_any(!ok || *abort_flag)) {
+      const int a = it % kAcc;
+      const bool ok = mbar_wait_bounded(accf0 + 8 * a, (uint32_t)(it / kAcc) & 1u);
+      // one decision per warp: tcgen05.ld below needs all 32 lanes
+      if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
+        if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
         *abort_flag = 1;
         break;
       }
       fence_after_sync();
-      const int rt = rt_first + it * row_step;
-      const int row = rt * kRows + r_local;
-      uint8_t* stage_out = smem + L.out_off + a * L.out_bytes;
-      uint8_t* stage_sc = smem + L.sc_off;
-      const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)a * acc_cols;
-      auto emit = [&](int jj, const float2 (&v)[16]) {
-        if constexpr (kTransformOnly) {
-          if (row < geo.M) {
-            float4* dst = reinterpret_cast<float4*>(y_out + ((size_t)row * nb + j0 + jj) * 32);
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-              dst[t] = make_float4(v[2 * t].x, v[2 * t].y, v[2 * t + 1].x, v[2 * t + 1].y);
-          }
-        } else {
-          uint4 packed;
-          const uint32_t byte = mxfp4_encode32(v, packed);
-          *reinterpret_cast<uint4*>(stage_out + out_offset(C, r_local, jj)) = packed;
-          stage_sc[r_local * C + jj] = (uint8_t)byte;
-        }
-      };
-      int jj = jj_lo;
-      for (; jj + 1 < jj_hi; jj += 2) {
-        float2 v0[16], v1[16];
-        tmem_ld32x2(tq + (uint32_t)(jj * 32), tq + (uint32_t)((jj + 1) * 32), v0, v1);
-        emit(jj, v0);
-        emit(jj + 1, v1);
-      }
-      if (jj < jj_hi) {
-        float2 v[16];
-        tmem_ld32(tq + (uint32_t)(jj * 32), v);
-        emit(jj, v);
+      const int64_t u = u_begin + it;
+      const int g = (int)(u / n_rt), rt = (int)(u - (int64_t)g * n_rt);
+      const int row = rt * kRows + 32 * q + lane;
+      const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * kAccCols);
+      float2 v0[16], v1[16];
+      const int cnt = jj_hi - jj_lo;
+      if (cnt == 2) {
+        tmem_ld32x2(tq + (uint32_t)(jj_lo * 32), tq + (uint32_t)((jj_lo + 1) * 32), v0, v1);
+      } else if (cnt == 1) {
+        tmem_ld32(tq + (uint32_t)(jj_lo * 32), v0);
       }
       // this warp's reads of accumulator a are complete: hand it back
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce0 + 8 * a);
-      if (!kTransformOnly) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        epi_barrier();
-        if (tid == 0) {
-          tma_store_2d(&omap, j0 * 16, rt * kRows, smem_addr(stage_out));
-          bulk_commit();
-        }
-        // scale bytes: consecutive threads write consecutive bytes of a row
-        for (int i = tid; i < kRows * C; i += kEpiWarps * 32) {
-          const int r = i / C, c = i - r * C;
-          const int grow = rt * kRows + r;
-          if (grow < geo.M) scales[(size_t)grow * nb + j0 + c] = stage_sc[i];
+      if (row < geo.M && cnt > 0) {
+        const size_t blk = (size_t)row * nb + (size_t)g * C + jj_lo;
+        uint4 p0, p1;
+        const uint32_t e0 = mxfp4_encode32(v0, p0);
+        *reinterpret_cast<uint4*>(codes + blk * 16) = p0;
+        if (cnt == 2) {
+          const uint32_t e1 = mxfp4_encode32(v1, p1);
+          *reinterpret_cast<uint4*>(codes + blk * 16 + 16) = p1;
+          if ((reinterpret_cast<uintptr_t>(scales + blk) & 1) == 0) {
+            *reinterpret_cast<uint16_t*>(scales + blk) = (uint16_t)(e0 | (e1 << 8));
+          } else {
+            scales[blk] = (uint8_t)e0;
+            scales[blk + 1] = (uint8_t)e1;
+          }
+        } else {
+          scales[blk] = (uint8_t)e0;
         }
       }
     }
-    if (!kTransformOnly && tid == 0) bulk_wait_all();
   }
 
   fence_before_sync();
@@ -425,6 +426,20 @@ int tc_choose_C(int nb) {
   return 1;
 }
 
+// Most column groups any CTA meets when U units are split into G balanced
+// contiguous ranges.
+int max_groups_met(int64_t U, int64_t G, int n_rt) {
+  int worst = 0;
+  for (int64_t i = 0; i < G; ++i) {
+    const int64_t b = i * U / G, e = (i + 1) * U / G;
+    if (e > b) {
+      const int span = (int)((e - 1) / n_rt - b / n_rt + 1);
+      if (span > worst) worst = span;
+    }
+  }
+  return worst;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tc_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -441,9 +456,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tc_encoder() {
 
 constexpr int kMaxDevices = 64;
 
-template <bool kTransformOnly>
-int tc_launch(const void* x, int64_t M, int64_t d, const float* params, uint8_t* codes,
-              uint8_t* scales, float* y, cudaStream_t stream) {
+}  // namespace
+
+int tc_quantize(const void* x, int64_t M, int64_t d, const float* params, uint8_t* codes,
+                uint8_t* scales, cudaStream_t stream) {
   TcGeometry geo;
   geo.nb = (int)(d / 32);
   geo.C = tc_choose_C(geo.nb);
@@ -452,7 +468,7 @@ int tc_launch(const void* x, int64_t M, int64_t d, const float* params, uint8_t*
   geo.n_row_tiles = (int)((M + tc::kRows - 1) / tc::kRows);
   const tc::Layout L = tc::layout_for(geo.C);
   const size_t smem = 1024 + (size_t)L.total;
-  auto kern = tc::tc_kernel<kTransformOnly>;
+  auto kern = tc::tc_kernel;
 
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -481,28 +497,14 @@ int tc_launch(const void* x, int64_t M, int64_t d, const float* params, uint8_t*
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
 
-  CUtensorMap om;
-  memset(&om, 0, sizeof(om));
-  if (!kTransformOnly) {
-    // codes [M][d/2] bytes; box = C*16 bytes x 128 rows
-    const cuuint64_t odims[2] = {(cuuint64_t)d / 2, (cuuint64_t)M};
-    const cuuint64_t ostrides[1] = {(cuuint64_t)d / 2};
-    const cuuint32_t obox[2] = {(cuuint32_t)(geo.C * 16), (cuuint32_t)tc::kRows};
-    const cuuint32_t oestr[2] = {1, 1};
-    const CUresult r2 = enc(&om, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, odims, ostrides, obox, oestr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            geo.C == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r2 != CUDA_SUCCESS)
-      return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled (codes) failed (CUresult %d)", (int)r2);
-  }
-
   int sms = 0;
   if (int st = sm_count(&sms)) return st;
-  int64_t per_group = sms / geo.NC;
-  if (per_group < 1) per_group = 1;
-  if (per_group > geo.n_row_tiles) per_group = geo.n_row_tiles;
-  const int64_t grid = per_group * geo.NC;
+  const int64_t U = (int64_t)geo.NC * geo.n_row_tiles;
+  int64_t grid = U < sms ? U : sms;
+  // every CTA keeps the T splits of the groups it meets: at most kMaxGroups
+  while (max_groups_met(U, grid, geo.n_row_tiles) > tc::kMaxGroups) grid += sms;
+  if (grid > U) grid = U;
+  if (grid > 0x7fffffff) return fail(KQ_ERR_UNSUPPORTED, "kq_quantize_tc: grid too large");
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -516,21 +518,9 @@ int tc_launch(const void* x, int64_t M, int64_t d, const float* params, uint8_t*
   cfg.numAttrs = 1;
   unsigned int* devstat = nullptr;
   if (int st = device_status_address(&devstat)) return st;
-  err = cudaLaunchKernelEx(&cfg, kern, tm, om, params, geo, codes, scales, y, devstat);
+  err = cudaLaunchKernelEx(&cfg, kern, tm, params, geo, codes, scales, devstat);
   if (err != cudaSuccess) return cuda_fail(err, "tc_kernel launch");
   return check_launch("tc_kernel launch");
-}
-
-}  // namespace
-
-int tc_quantize(const void* x, int64_t M, int64_t d, const float* params, uint8_t* codes,
-                uint8_t* scales, cudaStream_t stream) {
-  return tc_launch<false>(x, M, d, params, codes, scales, nullptr, stream);
-}
-
-int tc_transform(const void* x, int64_t M, int64_t d, const float* params, float* y,
-                 cudaStream_t stream) {
-  return tc_launch<true>(x, M, d, params, nullptr, nullptr, y, stream);
 }
 
 }  // namespace kq
