@@ -237,6 +237,59 @@ def ncu_traffic():
 
 
 # ---------------------------------------------------------------------------
+# weight side (offline, once per layer): fold + MXFP4 of the FLUX layer weights
+# ---------------------------------------------------------------------------
+WEIGHT_SHAPES = [(3072, 3072), (12288, 3072), (3072, 12288)]   # [N out][d in]
+
+
+def weight_bytes(N: int, d: int) -> float:
+    """fp32 weights read once, MXFP4 codes and scales written, 60 B of
+    parameters per block column."""
+    return N * d * (4 + 0.5 + 1 / 32) + (d // 32) * 60
+
+
+def time_weight_side(kq, device, stream, K: int, W: int) -> dict:
+    """kq_quantize_weights on the FLUX.1-schnell layer weight shapes: mean
+    device time of K back-to-back launches (each shape's weights are 38-151
+    MB, so a ring of 2 sets already exceeds L2)."""
+    import torch
+    lib = kq.abi()
+    peak, _ = hbm_peak()
+    out = {"kernel": "kq_quantize_weights (fold W T^-1 + MXFP4, fp32 in)", "shapes": {}}
+    for N, d in WEIGHT_SHAPES:
+        sets = []
+        for r in range(2):
+            Wt = torch.from_numpy(synthetic.make_weights(N, d, 20 + r)).to(device)
+            c = torch.empty((N, d // 2), dtype=torch.uint8, device=device)
+            sc = torch.empty((N, d // 32), dtype=torch.uint8, device=device)
+            sets.append((Wt, c, sc))
+        p = torch.from_numpy(synthetic.make_params(d // 32, 21)).to(device)
+
+        def go(k):
+            Wt, c, sc = sets[k % 2]
+            st = lib.kq_quantize_weights(Wt.data_ptr(), N, d, p.data_ptr(), c.data_ptr(),
+                                         sc.data_ptr(), stream.cuda_stream)
+            if st != 0:
+                raise RuntimeError(lib.kq_last_error().decode())
+        for k in range(W):
+            go(k)
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(K):
+            go(k)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) / K * 1e3
+        gbs = weight_bytes(N, d) / (us * 1e-6) / 1e9
+        out["shapes"][f"{N}x{d}"] = {"us": round(us, 2), "gbs": round(gbs, 1),
+                                     "frac_of_peak": round(gbs / peak, 4)}
+        del sets
+    return out
+
+
+# ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
 def run_kroquant(args) -> int:
@@ -380,6 +433,7 @@ def run_kroquant(args) -> int:
     launch_kq = [timed_burst(i, "kq", K, W) for i in range(len(rings))]
     launch_sq = [timed_burst(i, "sq", K, W) for i in range(len(rings))]
     launch_tc = timed_burst(dominant, "tc", K, W)
+    weight_side = time_weight_side(kq, device, stream, K, W)
 
     # end to end through the public API: pinned host input -> device -> quantize -> host
     host_out = [(torch.empty((w.M, w.d // 2), dtype=torch.uint8).pin_memory(),
@@ -487,6 +541,7 @@ def run_kroquant(args) -> int:
                 "gbs": round(dom_bytes / (launch_tc * 1e-3) / 1e9, 1),
                 "frac_of_peak": round(dom_bytes / (launch_tc * 1e-3) / 1e9 / peak, 4),
             },
+            "weight_side": weight_side,
             "e2e": {
                 "value": round(e2e_value, 2),
                 "unit": UNIT,

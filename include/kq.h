@@ -142,6 +142,21 @@ int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params,
                     float* W_out, void* stream);
 
 /*
+ * kq_quantize_weights -- the weight side of the W4A4 layer, done offline:
+ * the inverse transform folded into the weights (the abstract: the inverse
+ * goes to the weights) and the result quantised to MXFP4 like the
+ * activations, in 32-element blocks along d (the GEMM's reduction
+ * dimension, so weight and activation blocks line up).
+ *   W [N][d] fp32 (nn.Linear layout), params [d/32][15] as above.
+ *   codes [N][d/2] and scales [N][d/32]: the MXFP4 encoding (same rules as
+ *   kq_quantize) of W' = W blockdiag(T_j)^(-1), evaluated in fp32 exactly as
+ *   kq_fold_weights evaluates it; W' itself is never written.
+ *   W and codes 16-byte aligned, params 4-byte aligned.  Limit: N * d / 32 < 2^31.
+ */
+int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* params,
+                        uint8_t* codes, uint8_t* scales, void* stream);
+
+/*
  * kq_dequant -- MXFP4 back to fp32, for checking:
  *   out[m][c] = E2M1(code) * 2^(scale - 127); scale 0xFF gives NaN.
  *   codes [M][d/2] (16-byte aligned), scales [M][d/32], out [M][d] fp32

@@ -265,6 +265,14 @@ def fold_weights(W: np.ndarray, params: np.ndarray) -> np.ndarray:
     return out.reshape(n, d)
 
 
+def quantize_weights(W: np.ndarray, params: np.ndarray):
+    """[ABS] the weight side of the W4A4 layer: the folded weights
+    W' = W blockdiag(T_j)^{-1}, quantised to MXFP4 in 32-element blocks along
+    the input dimension d (the dimension the GEMM sums over, blocked like the
+    transformed activations).  Returns (codes [n, d/2], scales [n, d/32])."""
+    return quantize_mxfp4(fold_weights(W, params))
+
+
 def fold_error_scale(W: np.ndarray, params: np.ndarray) -> np.ndarray:
     """|W| times the magnitude of the inverse factors U^{-1} L^{-1}."""
     params = np.asarray(params).reshape(-1, PARAMS_PER_BLOCK)

@@ -334,6 +334,33 @@ def pin_fold_invariance(o):
     assert np.allclose(lhs, rhs, rtol=1e-10, atol=1e-10 * np.abs(rhs).max())
 
 
+def pin_weight_quantizer_direction(o):
+    """With a = b = 0 the transform is the diagonal D = diag(T), so the folded
+    weights are W D^{-1}: the weight codes equal plain MXFP4 of W divided
+    column-wise by diag(T), computed here without the oracle's fold; with
+    identity parameters they are plain MXFP4 of W."""
+    nb = 3
+    p = _rand_params(nb, seed=31).reshape(nb, 5, 3).copy()
+    p[:, :, 0] = 0
+    p[:, :, 1] = 0
+    p = p.reshape(nb, 15)
+    diag = np.empty(32 * nb)
+    for j in range(nb):
+        for i in range(32):
+            v = 1.0
+            for m in range(5):
+                u = p[j, 3 * m + 2]
+                v *= (1.0 / u) if (i >> (4 - m)) & 1 else u
+            diag[32 * j + i] = v
+    W = synthetic.make_weights(7, 32 * nb, 5).astype(np.float64)
+    c1, s1 = o.quantize_weights(W, p)
+    c2, s2 = o.quantize_mxfp4(W / diag[None, :])
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    ci, si = o.quantize_weights(W, synthetic.identity_params(nb))
+    c3, s3 = o.quantize_mxfp4(W)
+    assert np.array_equal(ci, c3) and np.array_equal(si, s3)
+
+
 def pin_smoothquant_is_diagonal_case(o):
     """a = b = 0 makes T diagonal; SmoothQuant with 1/s = diag(T) then gives
     the same codes and scales."""

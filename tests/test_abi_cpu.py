@@ -29,7 +29,8 @@ def header_functions():
 def test_header_declares_the_abi():
     names = header_functions()
     for want in ("kq_quantize", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
-                 "kq_fold_weights", "kq_dequant", "kq_status_string", "kq_device_status"):
+                 "kq_fold_weights", "kq_quantize_weights", "kq_dequant", "kq_status_string",
+                 "kq_device_status"):
         assert want in names
 
 
@@ -102,6 +103,11 @@ def test_other_argument_checks(lib):
     assert lib.kq_fold_weights(A16, 4, 64, A16b, A16 + 64, None) == 1   # partial overlap
     assert lib.kq_fold_weights(A16, 0, 64, A16b, A16c, None) == 0
     assert lib.kq_fold_weights(None, 0, 64, None, None, None) == 0
+    assert lib.kq_quantize_weights(A16, 4, 64, A16b, A16c + 8, A16d, None) == 2
+    assert lib.kq_quantize_weights(A16 + 4, 4, 64, A16b, A16c, A16d, None) == 2
+    assert lib.kq_quantize_weights(A16, 4, 48, A16b, A16c, A16d, None) == 1
+    assert lib.kq_quantize_weights(A16, 4, 64, None, A16c, A16d, None) == 1
+    assert lib.kq_quantize_weights(None, 0, 64, None, None, None, None) == 0
     assert lib.kq_dequant(A16, A16b, 4, 64, A16c + 4, None) == 2
     assert lib.kq_dequant(A16, A16b, 0, 64, A16c, None) == 0
     assert lib.kq_device_status(None, 0) == 1

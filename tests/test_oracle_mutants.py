@@ -134,6 +134,19 @@ def m_wrong_grid(o):
     o.E2M1_MAGNITUDES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 5.0])
 
 
+def m_weights_not_folded(o):
+    o.quantize_weights = lambda W, params: o.quantize_mxfp4(W)
+
+
+def m_weights_folded_with_forward(o):
+    def qw(W, params):
+        T = o.expand_params(params)
+        n, d = np.asarray(W).shape
+        Wb = np.asarray(W, dtype=np.float64).reshape(n, d // 32, 32)
+        return o.quantize_mxfp4(np.einsum("njk,jki->nji", Wb, T).reshape(n, d))
+    o.quantize_weights = qw
+
+
 MUTANTS = [v for k, v in sorted(globals().items()) if k.startswith("m_")]
 
 

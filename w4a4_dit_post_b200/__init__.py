@@ -20,7 +20,8 @@ from .build import LIB_PATH
 
 __all__ = [
     "abi", "kq_quantize", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
-    "kq_fold_weights", "kq_dequant", "kq_device_status", "kq_selftest_bounded_wait",
+    "kq_fold_weights", "kq_quantize_weights", "kq_dequant", "kq_device_status",
+    "kq_selftest_bounded_wait",
     "KroQuantError",
     "KQ_DTYPE_BF16", "KQ_DTYPE_F32", "KQ_MAX_D", "EXPORTED_FUNCTIONS",
 ]
@@ -42,6 +43,7 @@ _SIGNATURES = {
     "sq_quantize": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_expand_params": (_int, [_c_void_p, _i64, _c_void_p, _c_void_p]),
     "kq_fold_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "kq_quantize_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_dequant": (_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "kq_device_status": (_int, [ctypes.POINTER(ctypes.c_uint32), _int]),
     "kq_selftest_bounded_wait": (_int, [ctypes.c_uint32, _c_void_p]),
@@ -199,6 +201,20 @@ def kq_fold_weights(W, params, W_out=None):
         _check("kq_fold_weights", abi().kq_fold_weights(
             W.data_ptr(), N, d, params.data_ptr(), W_out.data_ptr(), _stream(W)))
     return W_out
+
+
+def kq_quantize_weights(W, params, codes=None, scales=None):
+    """Weight side: W [N, d] fp32 -> MXFP4 (codes uint8 [N, d/2], scales
+    uint8 [N, d/32]) of the folded weights W blockdiag(T_j)^{-1}."""
+    _need_cuda("W", W, (torch.float32,), 2)
+    _need_cuda("params", params, (torch.float32,))
+    N, d = W.shape
+    codes = _out(codes, (N, d // 2), torch.uint8, W, "codes")
+    scales = _out(scales, (N, d // 32), torch.uint8, W, "scales")
+    with torch.cuda.device(W.device):
+        _check("kq_quantize_weights", abi().kq_quantize_weights(
+            W.data_ptr(), N, d, params.data_ptr(), codes.data_ptr(), scales.data_ptr(), _stream(W)))
+    return codes, scales
 
 
 def kq_dequant(codes, scales, out=None):

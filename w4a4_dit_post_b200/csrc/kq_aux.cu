@@ -1,6 +1,6 @@
 // Support kernels: the dense blocks of the transform (kq_expand_params), the
-// inverse folded into the weights (kq_fold_weights) and MXFP4 decoding
-// (kq_dequant).  None of them is on the per-step path; they are simple,
+// inverse folded into the weights (kq_fold_weights), the folded weights
+// quantised to MXFP4 (kq_quantize_weights) and MXFP4 decoding (kq_dequant).  None of them is on the per-step path; they are simple,
 // memory-bound grid-stride kernels.
 #include <cuda_runtime.h>
 
@@ -57,6 +57,34 @@ fold_kernel(const float* W, const float* __restrict__ params, int nb, int n_bloc
 #pragma unroll
     for (int q = 0; q < 8; ++q)
       dst[q] = make_float4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
+  }
+}
+
+// Weight side: one thread per (weight row, block): the folded block
+// w T_j^{-1} (the same butterfly as fold_kernel) encoded to MXFP4 in
+// registers; the folded weights are never written.
+__global__ void __launch_bounds__(kAuxThreads)
+fold_quant_kernel(const float* __restrict__ W, const float* __restrict__ params, int nb,
+                  int n_blocks, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n_blocks; g += gridDim.x * blockDim.x) {
+    const int j = g % nb;
+    const float* p = params + 15 * j;
+    float4 B[5];
+#pragma unroll
+    for (int m = 0; m < 5; ++m) B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    const float4* src = reinterpret_cast<const float4*>(W + (size_t)g * 32);
+    float2 v[16];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 t = src[q];
+      v[2 * q] = make_float2(t.x, t.y);
+      v[2 * q + 1] = make_float2(t.z, t.w);
+    }
+    butterfly32(v, B);
+    uint4 packed;
+    const uint32_t byte = mxfp4_encode32(v, packed);
+    *reinterpret_cast<uint4*>(codes + (size_t)g * 16) = packed;
+    scales[g] = (uint8_t)byte;
   }
 }
 
@@ -142,6 +170,23 @@ int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params, f
   kq::fold_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
       W, params, nb, n_blocks, W_out);
   return kq::check_launch("fold_kernel launch");
+}
+
+int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* params,
+                        uint8_t* codes, uint8_t* scales, void* stream) {
+  if (int st = kq::check_shape(N, d, 0, "kq_quantize_weights")) return st;
+  if (N == 0) return KQ_OK;
+  if (!W || !params || !codes || !scales)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_weights: NULL pointer");
+  if (!kq::aligned(W, 16) || !kq::aligned(codes, 16))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_weights: W and codes must be 16-byte aligned");
+  if (!kq::aligned(params, 4))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_weights: params must be 4-byte aligned");
+  const int nb = (int)(d / 32);
+  const int n_blocks = (int)(N * nb);
+  kq::fold_quant_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+      W, params, nb, n_blocks, codes, scales);
+  return kq::check_launch("fold_quant_kernel launch");
 }
 
 int kq_dequant(const uint8_t* codes, const uint8_t* scales, int64_t M, int64_t d, float* out,
