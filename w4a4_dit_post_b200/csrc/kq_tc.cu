@@ -19,7 +19,8 @@
 // tcgen05.mma.
 //
 // Roles (320 threads):
-//   warp 8, lane 0: TMA producer (S shared-memory stages, S * C * 8 KiB <= 128 KiB);
+//   warp 8, lane 0: TMA producer (S shared-memory stages, S * C * 8 KiB <= 128 KiB,
+//                   plus an L2 prefetch of the unit S ahead);
 //   warp 9        : allocates tensor memory; lane 0 issues the MMAs:
 //                   per block column jj: 3 splits x 2 K-steps of
 //                   M=128 x N=32 x K=16 into accumulator columns jj*32..;
@@ -27,8 +28,12 @@
 //   warps 0..7    : epilogue.  Warp w reads TMEM lanes 32*(w%4).. (its token
 //                   rows) for half (w/4) of the unit's block columns with
 //                   tcgen05.ld 32x32b.x32 (one token's block per thread),
-//                   hands the accumulator back, and writes the MXFP4 codes
-//                   (16 bytes) and scale of each block straight to memory.
+//                   hands the accumulator back and encodes.  The unit's codes
+//                   are staged in shared memory (64-byte swizzle) and leave
+//                   by one TMA tensor store; its scale bytes leave row by row.
+//                   (The TMEM layout puts one token row in each thread, so
+//                   direct stores would scatter every warp's writes over 32
+//                   rows.)
 // Every mbarrier wait is bounded; a wait that runs out sets the device status
 // word and the CTA drains its copies and MMAs and exits.
 #include <cuda.h>
@@ -147,6 +152,9 @@ struct Layout {
   int stage_bytes;   // C * 128 * 64
   int table_off;     // kMaxGroups * C * 3 * 2048 bytes of T splits
   int fac_off;       // kMaxGroups * C * 5 float4 LU factors (set-up only)
+  int out_off;       // two code tiles of 128 rows x C * 16 bytes (TMA store sources)
+  int out_bytes;
+  int sc_off;        // two scale tiles of 128 rows x C bytes
   int bar_off;       // 2 S + 2 kAcc barriers, abort flag, TMEM address
   int total;
 };
@@ -158,13 +166,55 @@ __host__ __device__ inline Layout layout_for(int C) {
   if (L.stages > kMaxStages) L.stages = kMaxStages;
   L.table_off = L.stages * L.stage_bytes;
   L.fac_off = L.table_off + kMaxGroups * C * 3 * 2048;
-  L.bar_off = L.fac_off + 1024;
+  L.out_off = L.fac_off + 1024;
+  L.out_bytes = ((kRows * C * 16) + 1023) & ~1023;
+  L.sc_off = L.out_off + 2 * L.out_bytes;
+  L.bar_off = L.sc_off + 2 * kRows * kMaxC;
   L.total = L.bar_off + 512;
   return L;
 }
 
+// Staging position of (token row r, block jj) in a code tile of C*16-byte rows.
+// With C == 4 the rows are 64 bytes and the 64-byte swizzle (16-byte chunk ^=
+// (r >> 1) & 3) keeps a warp's 32 row writes free of bank conflicts; the TMA
+// store map uses the same swizzle.
+__device__ __forceinline__ int out_offset(int C, int r, int jj) {
+  return C == 4 ? r * 64 + ((jj ^ ((r >> 1) & 3)) << 4) : (r * C + jj) * 16;
+}
+
+__device__ __forceinline__ void tma_store_2d(const void* tmap, int c0, int c1, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Barrier 1 among the epilogue warps only (the producer and MMA warps never
+// take part).  epi_any also ORs a flag across them, so every epilogue warp
+// takes the same branch after it and no warp is left waiting.
+__device__ __forceinline__ void epi_barrier() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");
+}
+__device__ __forceinline__ bool epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(kEpiWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-tc_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ params,
+tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap omap,
+          const float* __restrict__ params,
           const TcGeometry geo, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
           unsigned int* devstat) {
   extern __shared__ uint8_t smem_raw[];
@@ -192,6 +242,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ pa
   pdl_launch_dependents();
   if (tid == 0) {
     tma_prefetch_desc(&tmap);
+    tma_prefetch_desc(&omap);
     for (int i = 0; i < S; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, 1);
@@ -230,8 +281,17 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ pa
     mbar_arrive_expect_tx(full0 + 8 * s, tx);
     tma_load_3d(smem_addr(smem + s * L.stage_bytes), &tmap, 0, rt * kRows, g * C, full0 + 8 * s);
   };
-  if (warp == kProducerWarp && lane == 0)
+  // L2 prefetch of a later unit: its bytes are on the way while the unit
+  // waits for a free stage, so more than the stages' worth is in flight
+  auto prefetch = [&](int it) {
+    const int64_t u = u_begin + it;
+    const int g = (int)(u / n_rt), rt = (int)(u - (int64_t)g * n_rt);
+    tma_prefetch_l2_3d(&tmap, 0, rt * kRows, g * C);
+  };
+  if (warp == kProducerWarp && lane == 0) {
     for (int it = 0; it < n_items && it < S; ++it) issue(it);
+    for (int it = S; it < n_items && it < 2 * S; ++it) prefetch(it);
+  }
 
   // T splits of the groups this CTA meets: [slot][jj][part][n = output row][k],
   // bf16, 64-byte rows with the 64-byte swizzle (16-byte chunk ^= (n >> 1) & 3).
@@ -302,6 +362,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ pa
         if (*abort_flag) break;
         issue(it);
         issued = it + 1;
+        if (it + S < n_items) prefetch(it + S);
       }
       // after an abort, let the copies still in flight land before the
       // shared memory goes away (on the normal path these return at once)
@@ -351,28 +412,31 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ pa
         (void)mbar_wait_bounded(accf0 + 8 * ((done - 1) % kAcc), (uint32_t)((done - 1) / kAcc) & 1u);
     }
   } else {
-    // epilogue warps: no barrier among them, so a warp that stops early
-    // leaves nobody waiting except through bounded mbarrier waits
+    // epilogue warps: the codes of a unit are staged in shared memory and
+    // written by one TMA tensor store (128 rows x C * 16 bytes), the scale
+    // bytes row by row; two staging buffers alternate
     const int q = warp & 3;                 // TMEM lane quarter = token rows 32q..32q+31
     const int h = warp >> 2;                // which half of the unit's block columns
     const int jj_lo = (h * C) / 2, jj_hi = ((h + 1) * C) / 2;
+    const int cnt = jj_hi - jj_lo;
     const int nb = geo.nb;
+    const int r_local = 32 * q + lane;      // token row inside the unit
     for (int it = 0; it < n_items; ++it) {
-      const int a = it % kAcc;
+      const int a = it % kAcc, buf = it & 1;
       const bool ok = mbar_wait_bounded(accf0 + 8 * a, (uint32_t)(it / kAcc) & 1u);
-      // one decision per warp: tcgen05.ld below needs all 32 lanes
-      if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
-        if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+      if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+      // the TMA store that last read this staging buffer (item it - 2) is done
+      if (tid == 0) bulk_wait_read_1();
+      // one decision for all epilogue warps (also the staging-buffer barrier)
+      if (epi_any(!ok || *abort_flag)) {
         *abort_flag = 1;
         break;
       }
       fence_after_sync();
       const int64_t u = u_begin + it;
       const int g = (int)(u / n_rt), rt = (int)(u - (int64_t)g * n_rt);
-      const int row = rt * kRows + 32 * q + lane;
       const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * kAccCols);
       float2 v0[16], v1[16];
-      const int cnt = jj_hi - jj_lo;
       if (cnt == 2) {
         tmem_ld32x2(tq + (uint32_t)(jj_lo * 32), tq + (uint32_t)((jj_lo + 1) * 32), v0, v1);
       } else if (cnt == 1) {
@@ -382,25 +446,40 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ pa
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce0 + 8 * a);
-      if (row < geo.M && cnt > 0) {
-        const size_t blk = (size_t)row * nb + (size_t)g * C + jj_lo;
-        uint4 p0, p1;
-        const uint32_t e0 = mxfp4_encode32(v0, p0);
-        *reinterpret_cast<uint4*>(codes + blk * 16) = p0;
+      uint8_t* stage_out = smem + L.out_off + buf * L.out_bytes;
+      uint8_t* stage_sc = smem + L.sc_off + buf * (kRows * kMaxC);
+      if (cnt > 0) {
+        uint4 p0;
+        stage_sc[r_local * C + jj_lo] = (uint8_t)mxfp4_encode32(v0, p0);
+        *reinterpret_cast<uint4*>(stage_out + out_offset(C, r_local, jj_lo)) = p0;
         if (cnt == 2) {
-          const uint32_t e1 = mxfp4_encode32(v1, p1);
-          *reinterpret_cast<uint4*>(codes + blk * 16 + 16) = p1;
-          if ((reinterpret_cast<uintptr_t>(scales + blk) & 1) == 0) {
-            *reinterpret_cast<uint16_t*>(scales + blk) = (uint16_t)(e0 | (e1 << 8));
+          uint4 p1;
+          stage_sc[r_local * C + jj_lo + 1] = (uint8_t)mxfp4_encode32(v1, p1);
+          *reinterpret_cast<uint4*>(stage_out + out_offset(C, r_local, jj_lo + 1)) = p1;
+        }
+      }
+      // generic-proxy writes -> visible to the TMA store, then all warps done
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      epi_barrier();
+      if (tid == 0) {
+        tma_store_2d(&omap, g * C * 16, rt * kRows, smem_addr(stage_out));
+        bulk_commit();
+      }
+      // scale bytes: one thread per token row writes the unit's C bytes
+      if (tid < kRows) {
+        const int row = rt * kRows + tid;
+        if (row < geo.M) {
+          uint8_t* dst = scales + (size_t)row * nb + (size_t)g * C;
+          const uint8_t* srcp = stage_sc + tid * C;
+          if (C == 4 && (reinterpret_cast<uintptr_t>(dst) & 3) == 0) {
+            *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(srcp);
           } else {
-            scales[blk] = (uint8_t)e0;
-            scales[blk + 1] = (uint8_t)e1;
+            for (int c = 0; c < C; ++c) dst[c] = srcp[c];
           }
-        } else {
-          scales[blk] = (uint8_t)e0;
         }
       }
     }
+    if (tid == 0) bulk_wait_all();
   }
 
   fence_before_sync();
@@ -497,6 +576,21 @@ int tc_quantize(const void* x, int64_t M, int64_t d, const float* params, uint8_
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
 
+  CUtensorMap om;
+  {
+    // codes [M][d/2] bytes; box = C*16 bytes x 128 rows
+    const cuuint64_t odims[2] = {(cuuint64_t)d / 2, (cuuint64_t)M};
+    const cuuint64_t ostrides[1] = {(cuuint64_t)d / 2};
+    const cuuint32_t obox[2] = {(cuuint32_t)(geo.C * 16), (cuuint32_t)tc::kRows};
+    const cuuint32_t oestr[2] = {1, 1};
+    const CUresult r2 = enc(&om, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, odims, ostrides, obox, oestr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            geo.C == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r2 != CUDA_SUCCESS)
+      return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled (codes) failed (CUresult %d)", (int)r2);
+  }
+
   int sms = 0;
   if (int st = sm_count(&sms)) return st;
   const int64_t U = (int64_t)geo.NC * geo.n_row_tiles;
@@ -518,7 +612,7 @@ int tc_quantize(const void* x, int64_t M, int64_t d, const float* params, uint8_
   cfg.numAttrs = 1;
   unsigned int* devstat = nullptr;
   if (int st = device_status_address(&devstat)) return st;
-  err = cudaLaunchKernelEx(&cfg, kern, tm, params, geo, codes, scales, devstat);
+  err = cudaLaunchKernelEx(&cfg, kern, tm, om, params, geo, codes, scales, devstat);
   if (err != cudaSuccess) return cuda_fail(err, "tc_kernel launch");
   return check_launch("tc_kernel launch");
 }
