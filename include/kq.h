@@ -12,6 +12,10 @@
  * Parameters (15 floats per block, fp32, layout [nb][15], nb = d / 32):
  *   factor m = 0..4 is (a, b, u) at [3m], [3m+1], [3m+2] and equals
  *   A = L U, L = [[1, 0], [a, 1]], U = [[u, b], [0, 1/u]]  (det A = 1).
+ *   u must be non-zero and a, b, u finite.  Every kernel that reads the
+ *   parameters checks this on the device: a violation sets
+ *   KQ_DEVSTAT_BAD_PARAMS in the status word (kq_device_status) and the
+ *   outputs of that call are unspecified; nothing faults.
  *   Factor m acts on bit (4 - m) of the channel index inside the block
  *   (factor 0 on the most significant bit: the standard Kronecker index map).
  *   Channel c = 32 j + i; y_j = T_j x_j for each token (column vector).
@@ -73,6 +77,7 @@ extern "C" {
 
 /* ---- device status bits (kq_device_status) -------------------------- */
 #define KQ_DEVSTAT_WAIT_TIMEOUT 0x1u   /* a bounded barrier wait ran out */
+#define KQ_DEVSTAT_BAD_PARAMS   0x2u   /* an LU factor had u == 0 or a non-finite a, b or u */
 
 /*
  * kq_quantize -- the online quantizer (the hot path).

@@ -1,4 +1,5 @@
-"""Failure detection without a GPU fault: a wait that runs out is reported in
+"""Failure detection without a GPU fault: a wait that runs out, or LU
+parameters that define no factor (u = 0, a non-finite value), are reported in
 the device status word, and the context stays usable.
 
 The self-test kernel waits on a barrier nothing arrives on (20 ms limit);
@@ -46,3 +47,39 @@ def test_timed_out_wait_is_reported_and_context_survives(kq):
 def test_selftest_argument_check(kq):
     with pytest.raises(RuntimeError):
         kq.kq_selftest_bounded_wait(0)
+
+
+def _bad_params(nb, where, value):
+    p = synthetic.make_params(nb, 3).copy()
+    p[where] = value
+    return torch.from_numpy(p).cuda()
+
+
+@pytest.mark.parametrize("where,value", [((1, 8), 0.0), ((0, 0), float("nan")), ((2, 4), float("inf"))],
+                         ids=["u_zero", "a_nan", "b_inf"])
+def test_bad_parameters_are_reported(kq, where, value):
+    """Every call that reads the LU parameters flags them; outputs are
+    unspecified, nothing faults, and good parameters afterwards are clean."""
+    M, d = 64, 96
+    nb = d // 32
+    pd = _bad_params(nb, where, value)
+    w = synthetic.Workload("badp", M, d, "bf16", "normal", 0.02, None, 20.0, 1.0, 8)
+    x = to_device(synthetic.make_activations(w), "bf16")
+    W = torch.from_numpy(synthetic.make_weights(16, d, 8)).cuda()
+    calls = [
+        lambda: kq.kq_quantize(x, pd),
+        lambda: kq.kq_quantize(x.float(), pd),
+        lambda: kq.kq_quantize_tc(x, pd),
+        lambda: kq.kq_transform(x, pd),
+        lambda: kq.kq_expand_params(pd),
+        lambda: kq.kq_fold_weights(W, pd),
+        lambda: kq.kq_quantize_weights(W, pd),
+    ]
+    assert kq.kq_device_status(clear=True) == 0
+    for call in calls:
+        call()
+        assert kq.kq_device_status(clear=True) == 0x2
+    good = torch.from_numpy(synthetic.make_params(nb, 3)).cuda()
+    for call in [lambda: kq.kq_quantize(x, good), lambda: kq.kq_quantize_weights(W, good)]:
+        call()
+        assert kq.kq_device_status() == 0

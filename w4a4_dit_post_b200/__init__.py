@@ -23,13 +23,16 @@ __all__ = [
     "kq_fold_weights", "kq_quantize_weights", "kq_dequant", "kq_device_status",
     "kq_selftest_bounded_wait",
     "KroQuantError",
-    "KQ_DTYPE_BF16", "KQ_DTYPE_F32", "KQ_MAX_D", "EXPORTED_FUNCTIONS",
+    "KQ_DTYPE_BF16", "KQ_DTYPE_F32", "KQ_MAX_D", "KQ_DEVSTAT_WAIT_TIMEOUT", "KQ_DEVSTAT_BAD_PARAMS",
+    "EXPORTED_FUNCTIONS",
 ]
 
 KQ_OK = 0
 KQ_DTYPE_BF16 = 0
 KQ_DTYPE_F32 = 1
 KQ_MAX_D = 32768
+KQ_DEVSTAT_WAIT_TIMEOUT = 0x1
+KQ_DEVSTAT_BAD_PARAMS = 0x2
 
 _c_void_p = ctypes.c_void_p
 _i64 = ctypes.c_int64

@@ -15,12 +15,14 @@ constexpr int kAuxThreads = 256;
 
 // T[j][i][k] = prod_m A_jm[bit(i, 4-m)][bit(k, 4-m)], one thread per entry.
 __global__ void __launch_bounds__(kAuxThreads)
-expand_kernel(const float* __restrict__ params, int nb, float* __restrict__ T) {
+expand_kernel(const float* __restrict__ params, int nb, float* __restrict__ T, unsigned int* devstat) {
   const int total = nb * 1024;
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += gridDim.x * blockDim.x) {
     const int j = idx >> 10, i = (idx >> 5) & 31, k = idx & 31;
     const float* p = params + 15 * j;
+    if ((idx & 1023) < 5 && lu_params_bad(p[3 * (idx & 1023)], p[3 * (idx & 1023) + 1], p[3 * (idx & 1023) + 2]))
+      atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
     float v = 1.0f;
 #pragma unroll
     for (int m = 0; m < 5; ++m) {
@@ -37,13 +39,19 @@ expand_kernel(const float* __restrict__ params, int nb, float* __restrict__ T) {
 // butterfly of the transposed inverse factors.  Reads the whole block before
 // writing it, so in-place use is safe.
 __global__ void __launch_bounds__(kAuxThreads)
-fold_kernel(const float* W, const float* __restrict__ params, int nb, int n_blocks, float* W_out) {
+fold_kernel(const float* W, const float* __restrict__ params, int nb, int n_blocks, float* W_out,
+            unsigned int* devstat) {
   for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n_blocks; g += gridDim.x * blockDim.x) {
     const int j = g % nb;
     const float* p = params + 15 * j;
     float4 B[5];
+    bool bad = false;
 #pragma unroll
-    for (int m = 0; m < 5; ++m) B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    for (int m = 0; m < 5; ++m) {
+      bad |= lu_params_bad(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+      B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    }
+    if (bad && g < nb) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
     const float4* src = reinterpret_cast<const float4*>(W + (size_t)g * 32);
     float2 v[16];
 #pragma unroll
@@ -65,13 +73,19 @@ fold_kernel(const float* W, const float* __restrict__ params, int nb, int n_bloc
 // registers; the folded weights are never written.
 __global__ void __launch_bounds__(kAuxThreads)
 fold_quant_kernel(const float* __restrict__ W, const float* __restrict__ params, int nb,
-                  int n_blocks, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+                  int n_blocks, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                  unsigned int* devstat) {
   for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n_blocks; g += gridDim.x * blockDim.x) {
     const int j = g % nb;
     const float* p = params + 15 * j;
     float4 B[5];
+    bool bad = false;
 #pragma unroll
-    for (int m = 0; m < 5; ++m) B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    for (int m = 0; m < 5; ++m) {
+      bad |= lu_params_bad(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+      B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    }
+    if (bad && g < nb) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
     const float4* src = reinterpret_cast<const float4*>(W + (size_t)g * 32);
     float2 v[16];
 #pragma unroll
@@ -145,8 +159,10 @@ int kq_expand_params(const float* params, int64_t d, float* T, void* stream) {
   const int64_t nb = d / 32;
   if (nb > (1 << 20)) return kq::fail(KQ_ERR_UNSUPPORTED, "kq_expand_params: d too large");
   const int total = (int)(nb * 1024);
+  unsigned int* devstat = nullptr;
+  if (int st = kq::device_status_address(&devstat)) return st;
   kq::expand_kernel<<<kq::grid_for(total), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
-      params, (int)nb, T);
+      params, (int)nb, T, devstat);
   return kq::check_launch("expand_kernel launch");
 }
 
@@ -167,8 +183,10 @@ int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params, f
   }
   const int nb = (int)(d / 32);
   const int n_blocks = (int)(N * nb);
+  unsigned int* devstat = nullptr;
+  if (int st = kq::device_status_address(&devstat)) return st;
   kq::fold_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
-      W, params, nb, n_blocks, W_out);
+      W, params, nb, n_blocks, W_out, devstat);
   return kq::check_launch("fold_kernel launch");
 }
 
@@ -184,8 +202,10 @@ int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* param
     return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_weights: params must be 4-byte aligned");
   const int nb = (int)(d / 32);
   const int n_blocks = (int)(N * nb);
+  unsigned int* devstat = nullptr;
+  if (int st = kq::device_status_address(&devstat)) return st;
   kq::fold_quant_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
-      W, params, nb, n_blocks, codes, scales);
+      W, params, nb, n_blocks, codes, scales, devstat);
   return kq::check_launch("fold_quant_kernel launch");
 }
 

@@ -167,6 +167,11 @@ __device__ __forceinline__ void butterfly32(float2 (&v)[16], const float4 (&A)[5
 }
 
 // Factor (A00, A01, A10, A11) of A = L U, L = [[1,0],[a,1]], U = [[u,b],[0,1/u]].
+// The factor is defined (and invertible) only for u != 0 and finite a, b, u.
+__device__ __forceinline__ bool lu_params_bad(float a, float b, float u) {
+  return u == 0.0f || !isfinite(a) || !isfinite(b) || !isfinite(u);
+}
+
 __device__ __forceinline__ float4 lu_factor(float a, float b, float u) {
   const float inv_u = 1.0f / u;
   return make_float4(u, b, __fmul_rn(a, u), __fmaf_rn(a, b, inv_u));

@@ -319,6 +319,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
     for (int i = tid; i < C * 5; i += kThreads) {
       const int cc = i / 5, m = i - 5 * cc;
       const float a = prm[15 * cc + 3 * m], b = prm[15 * cc + 3 * m + 1], u = prm[15 * cc + 3 * m + 2];
+      if (lu_params_bad(a, b, u)) atomicOr(&g_devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
       const float beta = b / u, gamma = __fmul_rn(__fmul_rn(a, u), u);
       *reinterpret_cast<float4*>(table + cc * kRow + 4 * m) = make_float4(beta, beta, gamma, gamma);
       uu[10 * cc + 2 * m] = u;

@@ -302,6 +302,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUte
   for (int i = tid; i < n_groups * C * 5; i += kThreads) {
     const int cj = i / 5, m = i - 5 * cj;   // cj = slot * C + jj
     const float* p = params + 15 * ((int64_t)g_first * C + cj) + 3 * m;
+    if (lu_params_bad(p[0], p[1], p[2])) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
     fac[i] = lu_factor(p[0], p[1], p[2]);
   }
   __syncthreads();
