@@ -70,35 +70,60 @@ fold_kernel(const float* W, const float* __restrict__ params, int nb, int n_bloc
 
 // Weight side: one thread per (weight row, block): the folded block
 // w T_j^{-1} (the same butterfly as fold_kernel) encoded to MXFP4 in
-// registers; the folded weights are never written.
+// registers; the folded weights are never written.  A warp takes 32
+// consecutive blocks (4 KiB of W): it reads them with coalesced 16-byte loads
+// into shared memory (16-byte chunk c of block b stored at chunk c ^ (b % 8),
+// so both the writes and the per-block reads are free of bank conflicts),
+// then every lane works on its own block; the codes of the 32 blocks leave
+// as 512 contiguous bytes, the scales as 32.
 __global__ void __launch_bounds__(kAuxThreads)
 fold_quant_kernel(const float* __restrict__ W, const float* __restrict__ params, int nb,
                   int n_blocks, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                   unsigned int* devstat) {
-  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n_blocks; g += gridDim.x * blockDim.x) {
-    const int j = g % nb;
-    const float* p = params + 15 * j;
-    float4 B[5];
-    bool bad = false;
+  __shared__ float4 stage[kAuxThreads / 32][32 * 8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4* st = stage[warp];
+  const int n_groups = (n_blocks + 31) / 32;
+  const int warps_total = gridDim.x * (blockDim.x >> 5);
+  for (int wg = blockIdx.x * (blockDim.x >> 5) + warp; wg < n_groups; wg += warps_total) {
+    const int g0 = wg * 32;
+    const int nblk = n_blocks - g0 < 32 ? n_blocks - g0 : 32;
+    const float4* src = reinterpret_cast<const float4*>(W + (size_t)g0 * 32);
 #pragma unroll
-    for (int m = 0; m < 5; ++m) {
-      bad |= lu_params_bad(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
-      B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    for (int i = 0; i < 8; ++i) {
+      const int L = lane + 32 * i;            // 16-byte chunk of the warp's 4 KiB
+      if (L < nblk * 8) {
+        const int b = L >> 3, c = L & 7;
+        st[b * 8 + (c ^ (b & 7))] = src[L];
+      }
     }
-    if (bad && g < nb) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
-    const float4* src = reinterpret_cast<const float4*>(W + (size_t)g * 32);
-    float2 v[16];
+    __syncwarp();
+    if (lane < nblk) {
+      const int g = g0 + lane;
+      const int j = g % nb;
+      const float* p = params + 15 * j;
+      float4 B[5];
+      bool bad = false;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 t = src[q];
-      v[2 * q] = make_float2(t.x, t.y);
-      v[2 * q + 1] = make_float2(t.z, t.w);
+      for (int m = 0; m < 5; ++m) {
+        bad |= lu_params_bad(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+        B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+      }
+      if (bad && g < nb) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
+      float2 v[16];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 t = st[lane * 8 + (q ^ (lane & 7))];
+        v[2 * q] = make_float2(t.x, t.y);
+        v[2 * q + 1] = make_float2(t.z, t.w);
+      }
+      butterfly32(v, B);
+      uint4 packed;
+      const uint32_t byte = mxfp4_encode32(v, packed);
+      *reinterpret_cast<uint4*>(codes + (size_t)g * 16) = packed;
+      scales[g] = (uint8_t)byte;
     }
-    butterfly32(v, B);
-    uint4 packed;
-    const uint32_t byte = mxfp4_encode32(v, packed);
-    *reinterpret_cast<uint4*>(codes + (size_t)g * 16) = packed;
-    scales[g] = (uint8_t)byte;
+    __syncwarp();
   }
 }
 
@@ -204,7 +229,9 @@ int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* param
   const int n_blocks = (int)(N * nb);
   unsigned int* devstat = nullptr;
   if (int st = kq::device_status_address(&devstat)) return st;
-  kq::fold_quant_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+  // one warp per 32 blocks
+  const int64_t lanes = (int64_t)((n_blocks + 31) / 32) * 32;
+  kq::fold_quant_kernel<<<kq::grid_for((int)lanes), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
       W, params, nb, n_blocks, codes, scales, devstat);
   return kq::check_launch("fold_quant_kernel launch");
 }
