@@ -162,6 +162,32 @@ int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* param
                         uint8_t* codes, uint8_t* scales, void* stream);
 
 /*
+ * kq_sf_tile -- scale bytes in the blocked layout the tensor cores read them
+ * from (the operand format of kq_gemm_mxfp4; no page counterpart: a layout
+ * of the hardware).
+ *   scales [R][K/32] uint8 row-major (as written by kq_quantize or
+ *   kq_quantize_weights) -> tiled [ceil(R/128)][K/128][512] uint8: row r and
+ *   scale column s at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + s % 4 of
+ *   block (r / 128, s / 4); rows past R are zero.  K a multiple of 128.
+ */
+int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void* stream);
+
+/*
+ * kq_gemm_mxfp4 -- the W4A4 linear layer on the quantised operands (the step
+ * after the quantizer: "before quantizing both" weights and activations to 4
+ * bits, the abstract):
+ *   Y[m][n] = sum_k a[m][k] * b[n][k], a = the MXFP4 activations (codes
+ *   [M][K/2] from kq_quantize, scales tiled by kq_sf_tile), b = the MXFP4
+ *   folded weights (codes [N][K/2] from kq_quantize_weights, scales tiled).
+ *   Y [M][N] fp32 row-major.  Products on the tensor cores with the
+ *   block-scaled FP4 MMA, fp32 accumulation in tensor memory.
+ *   K a multiple of 128; all pointers 16-byte aligned; ceil(M/128) <= 65535.
+ */
+int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                  const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, float* Y,
+                  void* stream);
+
+/*
  * kq_dequant -- MXFP4 back to fp32, for checking:
  *   out[m][c] = E2M1(code) * 2^(scale - 127); scale 0xFF gives NaN.
  *   codes [M][d/2] (16-byte aligned), scales [M][d/32], out [M][d] fp32

@@ -273,6 +273,38 @@ def quantize_weights(W: np.ndarray, params: np.ndarray):
     return quantize_mxfp4(fold_weights(W, params))
 
 
+def gemm_mxfp4(codes_a, scales_a, codes_b, scales_b) -> np.ndarray:
+    """[ABS] the W4A4 linear layer on the quantised operands: every MXFP4
+    value decoded (E2M1 code times its block's E8M0 scale), then
+    Y = A B^T summed over the input dimension in fp64, where A [M, K] are the
+    activation codes and B [N, K] the weight codes."""
+    return dequant(codes_a, scales_a) @ dequant(codes_b, scales_b).T
+
+
+def gemm_error_scale(codes_a, scales_a, codes_b, scales_b) -> np.ndarray:
+    """sum_k |a_k| |b_k| per output: the size of the terms an fp32
+    accumulation adds up."""
+    return np.abs(dequant(codes_a, scales_a)) @ np.abs(dequant(codes_b, scales_b)).T
+
+
+def sf_tile(scales: np.ndarray) -> np.ndarray:
+    """Scale bytes [R, K/32] (row-major) in the blocked layout the tensor
+    cores read scale factors from: for each 128-row tile and each group of 4
+    scale columns (128 input channels), 512 bytes in which row r of the tile
+    and scale column j of the group sit at byte (r % 32) * 16 + (r // 32) * 4 + j.
+    Rows beyond R are padded to a multiple of 128 with zero bytes.  Returns a
+    flat uint8 array [ceil(R/128), (K/32)/4, 512]."""
+    scales = np.asarray(scales, dtype=np.uint8)
+    R, ns = scales.shape
+    assert ns % 4 == 0
+    rt = (R + 127) // 128
+    out = np.zeros((rt, ns // 4, 512), dtype=np.uint8)
+    for r in range(R):
+        for s in range(ns):
+            out[r // 128, s // 4, (r % 32) * 16 + ((r % 128) // 32) * 4 + (s % 4)] = scales[r, s]
+    return out
+
+
 def fold_error_scale(W: np.ndarray, params: np.ndarray) -> np.ndarray:
     """|W| times the magnitude of the inverse factors U^{-1} L^{-1}."""
     params = np.asarray(params).reshape(-1, PARAMS_PER_BLOCK)

@@ -361,6 +361,36 @@ def pin_weight_quantizer_direction(o):
     assert np.array_equal(ci, c3) and np.array_equal(si, s3)
 
 
+def pin_gemm_mxfp4_by_hand(o):
+    """The quantised GEMM against a plain triple loop over decoded values,
+    each decoded by hand from the E2M1 grid and 2**(byte - 127); and the
+    blocked scale layout against its defining formula on a small case."""
+    rng = np.random.default_rng(41)
+    M, N, K = 3, 2, 64
+    ca = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    cb = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sa = rng.integers(120, 135, size=(M, K // 32), dtype=np.uint8)
+    sb = rng.integers(120, 135, size=(N, K // 32), dtype=np.uint8)
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+    def val(codes, scales, r, k):
+        byte = int(codes[r, k // 2])
+        nib = (byte >> 4) if k % 2 else (byte & 15)
+        mag = grid[nib & 7] * 2.0 ** (int(scales[r, k // 32]) - 127)
+        return -mag if nib & 8 else mag
+    Y = o.gemm_mxfp4(ca, sa, cb, sb)
+    for m in range(M):
+        for n in range(N):
+            ref = math.fsum(val(ca, sa, m, k) * val(cb, sb, n, k) for k in range(K))
+            assert Y[m, n] == ref
+    sc = np.arange(130 * 8, dtype=np.uint32).reshape(130, 8).astype(np.uint8)
+    t = o.sf_tile(sc)
+    assert t.shape == (2, 2, 512)
+    assert t[0, 0, 0] == sc[0, 0] and t[0, 0, 1] == sc[0, 1] and t[0, 0, 4] == sc[32, 0]
+    assert t[0, 1, 16 * 5 + 4 * 3 + 2] == sc[101, 6]
+    assert t[1, 1, 16 * 1 + 3] == sc[129, 7] and t[1, 0, 16 * 2] == 0
+
+
 def pin_smoothquant_is_diagonal_case(o):
     """a = b = 0 makes T diagonal; SmoothQuant with 1/s = diag(T) then gives
     the same codes and scales."""

@@ -1,0 +1,92 @@
+"""The W4A4 GEMM on the quantised operands (kq_sf_tile + kq_gemm_mxfp4)
+against the oracle.  Operand codes and scales are seeded or come from the
+oracle's own quantizers; the GPU computes Y from them.  Needs a B200.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.kq_oracle as o
+import synthetic
+from gpu_util import f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kq():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from w4a4_dit_post_b200 import build
+    build.build()
+    import w4a4_dit_post_b200 as k
+    k.kq_device_status(clear=True)
+    yield k
+    assert k.kq_device_status() == 0, "a bounded device wait ran out"
+
+
+def _cuda(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _operands(rng, rows, K, scale_lo, scale_hi):
+    codes = rng.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+    scales = rng.integers(scale_lo, scale_hi + 1, size=(rows, K // 32), dtype=np.uint8)
+    return codes, scales
+
+
+def _gemm(kq, ca, sa, cb, sb):
+    ta = kq.kq_sf_tile(_cuda(sa))
+    tb = kq.kq_sf_tile(_cuda(sb))
+    Y = kq.kq_gemm_mxfp4(_cuda(ca), ta, _cuda(cb), tb)
+    torch.cuda.synchronize()
+    return Y.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("R,K", [(1, 128), (130, 256), (4608, 3072)])
+def test_sf_tile_matches_oracle(kq, R, K):
+    rng = np.random.default_rng(R + K)
+    s = rng.integers(0, 256, size=(R, K // 32), dtype=np.uint8)
+    t = kq.kq_sf_tile(_cuda(s)).cpu().numpy()
+    assert np.array_equal(t, o.sf_tile(s))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (200, 72, 384), (256, 384, 1024), (1, 1, 128)])
+def test_gemm_unit_scales_is_exact(kq, M, N, K):
+    """Unit scales: every product is a multiple of 1/4 below 36 and every sum
+    fits fp32 exactly, so any accumulation order gives the oracle's bits.  A
+    misplaced code, scale or row shows up as a wrong value."""
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    ca, sa = _operands(rng, M, K, 127, 127)
+    cb, sb = _operands(rng, N, K, 127, 127)
+    Y = _gemm(kq, ca, sa, cb, sb)
+    assert np.array_equal(Y, o.gemm_mxfp4(ca, sa, cb, sb))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (200, 72, 384), (384, 256, 3072)])
+def test_gemm_scaled_operands(kq, M, N, K):
+    """Scales 2^-10 .. 2^10 per 32-element block (each block of each row its
+    own): within fp32 accumulation error of the fp64 product."""
+    rng = np.random.default_rng(M + 11 * N + K)
+    ca, sa = _operands(rng, M, K, 117, 137)
+    cb, sb = _operands(rng, N, K, 117, 137)
+    Y = _gemm(kq, ca, sa, cb, sb)
+    ref = o.gemm_mxfp4(ca, sa, cb, sb)
+    tol = (K / 64 + 64) * 2.0 ** -23 * o.gemm_error_scale(ca, sa, cb, sb)
+    assert np.all(np.abs(Y - ref) <= tol)
+
+
+def test_gemm_on_quantized_layer(kq):
+    """A FLUX.1-schnell-shaped layer: 512 tokens x 3072 channels through the
+    oracle's KroQuant quantizer, 256 x 3072 weights through the oracle's
+    weight quantizer (folded), then the GPU GEMM on those codes."""
+    w = synthetic.CONFIGS["flux"][0]
+    X = f64(synthetic.make_activations(w, np.arange(512)), w.dtype)
+    W = synthetic.make_weights(256, w.d, 10).astype(np.float64)
+    p = synthetic.make_params(w.nb, w.seed)
+    ca, sa = o.kq_quantize(X, p)
+    cb, sb = o.quantize_weights(W, p)
+    Y = _gemm(kq, ca, sa, cb, sb)
+    ref = o.gemm_mxfp4(ca, sa, cb, sb)
+    tol = (w.d / 64 + 64) * 2.0 ** -23 * o.gemm_error_scale(ca, sa, cb, sb)
+    assert np.all(np.abs(Y - ref) <= tol)

@@ -20,7 +20,8 @@ from .build import LIB_PATH
 
 __all__ = [
     "abi", "kq_quantize", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
-    "kq_fold_weights", "kq_quantize_weights", "kq_dequant", "kq_device_status",
+    "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4", "kq_dequant",
+    "kq_device_status",
     "kq_selftest_bounded_wait",
     "KroQuantError",
     "KQ_DTYPE_BF16", "KQ_DTYPE_F32", "KQ_MAX_D", "KQ_DEVSTAT_WAIT_TIMEOUT", "KQ_DEVSTAT_BAD_PARAMS",
@@ -47,6 +48,9 @@ _SIGNATURES = {
     "kq_expand_params": (_int, [_c_void_p, _i64, _c_void_p, _c_void_p]),
     "kq_fold_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
     "kq_quantize_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "kq_sf_tile": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
+    "kq_gemm_mxfp4": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _c_void_p,
+                             _c_void_p]),
     "kq_dequant": (_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "kq_device_status": (_int, [ctypes.POINTER(ctypes.c_uint32), _int]),
     "kq_selftest_bounded_wait": (_int, [ctypes.c_uint32, _c_void_p]),
@@ -218,6 +222,42 @@ def kq_quantize_weights(W, params, codes=None, scales=None):
         _check("kq_quantize_weights", abi().kq_quantize_weights(
             W.data_ptr(), N, d, params.data_ptr(), codes.data_ptr(), scales.data_ptr(), _stream(W)))
     return codes, scales
+
+
+def kq_sf_tile(scales, out=None):
+    """Scale bytes [R, K/32] -> the blocked layout [ceil(R/128), K/128, 512]
+    that kq_gemm_mxfp4 reads."""
+    _need_cuda("scales", scales, (torch.uint8,), 2)
+    R, ns = scales.shape
+    K = 32 * ns
+    out = _out(out, ((R + 127) // 128, K // 128 if K % 128 == 0 else 0, 512), torch.uint8, scales, "out")
+    with torch.cuda.device(scales.device):
+        _check("kq_sf_tile", abi().kq_sf_tile(scales.data_ptr(), R, K, out.data_ptr(), _stream(scales)))
+    return out
+
+
+def kq_gemm_mxfp4(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
+    """Y [M, N] fp32 = MXFP4(A) MXFP4(B)^T from codes [M, K/2] / [N, K/2] and
+    scales tiled by kq_sf_tile."""
+    for name, t in (("a_codes", a_codes), ("b_codes", b_codes)):
+        _need_cuda(name, t, (torch.uint8,), 2)
+    for name, t in (("a_sf_tiled", a_sf_tiled), ("b_sf_tiled", b_sf_tiled)):
+        _need_cuda(name, t, (torch.uint8,), 3)
+    M, half = a_codes.shape
+    N = b_codes.shape[0]
+    K = 2 * half
+    if b_codes.shape[1] != half:
+        raise ValueError("a_codes and b_codes disagree on K")
+    for name, t, rows in (("a_sf_tiled", a_sf_tiled, M), ("b_sf_tiled", b_sf_tiled, N)):
+        if tuple(t.shape) != ((rows + 127) // 128, K // 128, 512):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected "
+                             f"{((rows + 127) // 128, K // 128, 512)}")
+    Y = _out(Y, (M, N), torch.float32, a_codes, "Y")
+    with torch.cuda.device(a_codes.device):
+        _check("kq_gemm_mxfp4", abi().kq_gemm_mxfp4(
+            a_codes.data_ptr(), a_sf_tiled.data_ptr(), b_codes.data_ptr(), b_sf_tiled.data_ptr(),
+            M, N, K, Y.data_ptr(), _stream(a_codes)))
+    return Y
 
 
 def kq_dequant(codes, scales, out=None):

@@ -1,0 +1,397 @@
+// The W4A4 linear layer on the quantised operands: Y = A B^T, where A [M, K]
+// are MXFP4 activation codes (kq_quantize) and B [N, K] MXFP4 weight codes
+// (kq_quantize_weights), each with one E8M0 scale per 32 values along K.
+//
+// The products run on the 5th-generation tensor cores with the block-scaled
+// FP4 MMA (tcgen05.mma kind::mxf4, one scale per 32 elements): the E2M1 codes
+// go in as stored (two per byte), the scales ride along in tensor memory, and
+// the fp32 accumulator lives in tensor memory.
+//
+// Scale factors.  The MMA reads the scale of row m from tensor-memory lane m,
+// column m / 32 of a 4-column group, byte = scale index within a group of
+// four.  A 512-byte block of shared memory holding, for 128 rows and 4 scale
+// columns, row r's 4 scales at byte (r % 32) * 16 + (r / 32) * 4 becomes
+// exactly that group through one tcgen05.cp 32x128b.warpx4 (32 lanes x 16
+// bytes, copied into all four lane quarters).  kq_sf_tile rewrites the
+// row-major scale bytes into such 512-byte blocks once per operand.
+//
+// Tiling.  One CTA computes a 128 x 128 tile of Y; K advances in steps of 128
+// (64 bytes of codes per row, 4 scales): per step one TMA load of A and of B
+// (128 rows x 64 bytes, 64-byte swizzle: the canonical K-major operand
+// layout), one bulk copy of each 512-byte scale block, two MMAs of K = 64.
+// Roles (192 threads): warp 0 lane 0 loads (S stages), warp 1 owns tensor
+// memory and lane 0 issues the scale copies and MMAs, warps 2..5 read the
+// accumulator (one row per thread) and store fp32 rows.  Every wait is
+// bounded; a wait that runs out sets the device status word and the CTA
+// drains and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "kq.h"
+#include "kq_device.cuh"
+#include "kq_host.h"
+
+namespace kq {
+namespace gemm {
+
+constexpr int kThreads = 192;
+constexpr int kTile = 128;          // M and N of the CTA tile (and of the MMA)
+constexpr int kKStep = 128;         // K per stage (fp4 elements)
+constexpr int kStages = 6;
+constexpr int kOpBytes = kTile * kKStep / 2;        // 8 KiB of codes per operand per stage
+constexpr int kSfBytes = 512;
+constexpr int kStageBytes = 2 * kOpBytes + 2 * kSfBytes;
+constexpr int kTmemCols = 256;      // 128 accumulator columns + 8 scale columns
+constexpr int kSfaCol = 128, kSfbCol = 132;
+
+// Block-scaled instruction descriptor: A, B = E2M1 (MXF4), scales E8M0,
+// both K-major, N = 128, M = 128, K = 64; the scale-factor ids go in bits
+// 29-30 (A) and 4-5 (B).
+constexpr uint32_t kIdescBase = (1u << 7) | (1u << 10) | ((uint32_t)(kTile >> 3) << 17) | (1u << 23) |
+                                ((uint32_t)(kTile >> 4) << 24);
+
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(512 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)4 << 61);
+}
+
+// Descriptor of one 512-byte scale block as the source of tcgen05.cp:
+// 32 rows of 16 bytes, no swizzle, 8-row groups 128 bytes apart.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t sfa, uint32_t sfb, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 1-D bulk copy global -> shared, completion on an mbarrier (16-byte aligned).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+struct GemmArgs {
+  int M, N, K;
+  int k_steps;               // K / 128
+  const uint8_t* sfa;        // blocked scales of A: [ceil(M/128)][K/128][512]
+  const uint8_t* sfb;        // blocked scales of B
+  float* Y;                  // [M][N] fp32
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+            const GemmArgs args, unsigned int* devstat) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kStages]);
+  const uint32_t accf = smem_addr(&bars[2 * kStages]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 1));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 2));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_tile = blockIdx.x, m_tile = blockIdx.y;
+  const int KS = args.k_steps;
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&bmap);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait_predecessor();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint8_t* sfa_tile = args.sfa + (size_t)m_tile * KS * kSfBytes;
+      const uint8_t* sfb_tile = args.sfb + (size_t)n_tile * KS * kSfBytes;
+      int issued = 0;
+      for (int kt = 0; kt < KS; ++kt) {
+        const int s = kt % kStages;
+        if (kt >= kStages && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(kt / kStages - 1) & 1u)) {
+          *abort_flag = 1;
+          atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+          break;
+        }
+        if (*abort_flag) break;
+        uint8_t* st = smem + s * kStageBytes;
+        const uint32_t bar = full0 + 8 * s;
+        mbar_arrive_expect_tx(bar, (uint32_t)kStageBytes);
+        tma_load_2d(smem_addr(st), &amap, kt * (kKStep / 2), m_tile * kTile, bar);
+        tma_load_2d(smem_addr(st + kOpBytes), &bmap, kt * (kKStep / 2), n_tile * kTile, bar);
+        bulk_load(smem_addr(st + 2 * kOpBytes), sfa_tile + (size_t)kt * kSfBytes, kSfBytes, bar);
+        bulk_load(smem_addr(st + 2 * kOpBytes + kSfBytes), sfb_tile + (size_t)kt * kSfBytes, kSfBytes, bar);
+        issued = kt + 1;
+      }
+      if (*abort_flag) {
+        const int lo = issued > kStages ? issued - kStages : 0;
+        for (int kt = lo; kt < issued; ++kt)
+          (void)mbar_wait_bounded(full0 + 8 * (kt % kStages), (uint32_t)(kt / kStages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool issued_any = false;
+      for (int kt = 0; kt < KS; ++kt) {
+        const int s = kt % kStages;
+        if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)(kt / kStages) & 1u) || *abort_flag) {
+          *abort_flag = 1;
+          atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+          break;
+        }
+        fence_after_sync();
+        const uint32_t st = smem_addr(smem + s * kStageBytes);
+        // scale blocks of this step into tensor memory (in issue order with
+        // the MMAs below, and after the MMAs of the previous step)
+        sf_copy(tmem_base + kSfaCol, sf_desc(st + 2 * kOpBytes));
+        sf_copy(tmem_base + kSfbCol, sf_desc(st + 2 * kOpBytes + kSfBytes));
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t sf_id = (uint32_t)(2 * kk);      // scales 2kk, 2kk+1 of the group of 4
+          const uint32_t sfa = (tmem_base + kSfaCol) | (sf_id << 30);
+          const uint32_t sfb = (tmem_base + kSfbCol) | (sf_id << 30);
+          const uint32_t idesc = kIdescBase | (sf_id << 29) | (sf_id << 4);
+          mma_mxf4(tmem_base, sw64_desc(st + kk * 32), sw64_desc(st + kOpBytes + kk * 32), idesc,
+                   sfa, sfb, (kt | kk) != 0);
+        }
+        mma_commit(empty0 + 8 * s);
+        issued_any = true;
+      }
+      if (!*abort_flag) {
+        mma_commit(accf);
+      } else if (issued_any) {
+        // let the MMAs already issued finish before tensor memory is freed
+        mma_commit(accf);
+        (void)mbar_wait_bounded(accf, 0);
+      }
+    }
+  } else {
+    // epilogue: warps 2..5 -> TMEM lane quarters (warp % 4)
+    const int q = warp & 3;
+    const int row = m_tile * kTile + 32 * q + lane;
+    const bool ok = mbar_wait_bounded(accf, 0);
+    if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
+      if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+    } else {
+      fence_after_sync();
+      const int n0 = n_tile * kTile;
+      for (int c = 0; c < kTile / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+        if (row < args.M) {
+          float* dst = args.Y + (size_t)row * args.N + n0 + 32 * c;
+          const int n_valid = args.N - (n0 + 32 * c);
+          if (n_valid >= 32 && (args.N & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              reinterpret_cast<float4*>(dst)[i] =
+                  make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                              __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          } else {
+            for (int i = 0; i < 32 && i < n_valid; ++i) dst[i] = __uint_as_float(r[i]);
+          }
+        }
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// Row-major scale bytes [R][K/32] -> 512-byte blocks [ceil(R/128)][K/128][512]
+// (row r, scale column s at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + s % 4
+// of block (r / 128, s / 4)); rows past R become zero.  One thread per output byte.
+__global__ void __launch_bounds__(256)
+sf_tile_kernel(const uint8_t* __restrict__ scales, int R, int ns, int n_out, uint8_t* __restrict__ out) {
+  for (int o = blockIdx.x * blockDim.x + threadIdx.x; o < n_out; o += gridDim.x * blockDim.x) {
+    const int blk = o >> 9, within = o & 511;
+    const int groups = ns >> 2;
+    const int rt = blk / groups, g = blk - rt * groups;
+    const int r0 = within >> 4, r1 = (within >> 2) & 3, j = within & 3;
+    const int r = rt * 128 + r1 * 32 + r0;
+    out[o] = r < R ? scales[(size_t)r * ns + 4 * g + j] : (uint8_t)0;
+  }
+}
+
+}  // namespace gemm
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 gemm_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int codes_tmap(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t K) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = gemm_encoder();
+  if (!enc) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled not found in the CUDA driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+  const cuuint32_t box[2] = {gemm::kKStep / 2, gemm::kTile};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return KQ_OK;
+}
+
+constexpr int kMaxDevices = 64;
+
+}  // namespace
+}  // namespace kq
+
+extern "C" {
+
+int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void* stream) {
+  const char* fn = "kq_sf_tile";
+  if (R < 0 || K <= 0 || K % 128 != 0)
+    return kq::fail(KQ_ERR_INVALID_ARG, "%s: need R >= 0 and K a positive multiple of 128 (K = %lld)", fn,
+                    (long long)K);
+  if (R == 0) return KQ_OK;
+  if (!scales || !tiled) return kq::fail(KQ_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  const int64_t n_out = (R + 127) / 128 * (K / 128) * 512;
+  if (n_out >= ((int64_t)1 << 31) || R * (K / 32) >= ((int64_t)1 << 31))
+    return kq::fail(KQ_ERR_UNSUPPORTED, "%s: too large", fn);
+  int sms = 0;
+  if (int st = kq::sm_count(&sms)) return st;
+  int64_t blocks = (n_out + 255) / 256;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  kq::gemm::sf_tile_kernel<<<(unsigned)blocks, 256, 0, kq::as_stream(stream)>>>(
+      scales, (int)R, (int)(K / 32), (int)n_out, tiled);
+  return kq::check_launch("sf_tile_kernel launch");
+}
+
+int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                  const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, float* Y, void* stream) {
+  const char* fn = "kq_gemm_mxfp4";
+  if (M < 0 || N < 0 || K <= 0 || K % 128 != 0)
+    return kq::fail(KQ_ERR_INVALID_ARG, "%s: need M, N >= 0 and K a positive multiple of 128", fn);
+  if (M == 0 || N == 0) return KQ_OK;
+  if (!a_codes || !a_sf_tiled || !b_codes || !b_sf_tiled || !Y)
+    return kq::fail(KQ_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!kq::aligned(a_codes, 16) || !kq::aligned(b_codes, 16) || !kq::aligned(a_sf_tiled, 16) ||
+      !kq::aligned(b_sf_tiled, 16) || !kq::aligned(Y, 16))
+    return kq::fail(KQ_ERR_ALIGNMENT, "%s: codes, tiled scales and Y must be 16-byte aligned", fn);
+  if ((M + 127) / 128 > 65535 || N >= ((int64_t)1 << 31) / 128 || K >= ((int64_t)1 << 24) ||
+      M * N >= ((int64_t)1 << 40))
+    return kq::fail(KQ_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", fn);
+
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return kq::cuda_fail(err, "cudaGetDevice");
+  if (dev < 0 || dev >= kq::kMaxDevices) return kq::fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  const size_t smem = 1024 + (size_t)kq::gemm::kStages * kq::gemm::kStageBytes + 256;
+  static std::once_flag attr_once[kq::kMaxDevices];
+  static cudaError_t attr_err[kq::kMaxDevices];
+  std::call_once(attr_once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  });
+  if (attr_err[dev] != cudaSuccess) return kq::cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
+
+  CUtensorMap am, bm;
+  if (int st = kq::codes_tmap(&am, a_codes, M, K)) return st;
+  if (int st = kq::codes_tmap(&bm, b_codes, N, K)) return st;
+  kq::gemm::GemmArgs args;
+  args.M = (int)M;
+  args.N = (int)N;
+  args.K = (int)K;
+  args.k_steps = (int)(K / kq::gemm::kKStep);
+  args.sfa = a_sf_tiled;
+  args.sfb = b_sf_tiled;
+  args.Y = Y;
+  unsigned int* devstat = nullptr;
+  if (int st = kq::device_status_address(&devstat)) return st;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((N + 127) / 128), (unsigned)((M + 127) / 128));
+  cfg.blockDim = dim3(kq::gemm::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = kq::as_stream(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel, am, bm, args, devstat);
+  if (err != cudaSuccess) return kq::cuda_fail(err, "gemm_kernel launch");
+  return kq::check_launch("gemm_kernel launch");
+}
+
+}  // extern "C"
