@@ -290,6 +290,63 @@ def time_weight_side(kq, device, stream, K: int, W: int) -> dict:
 
 
 # ---------------------------------------------------------------------------
+# the layer's GEMM on the quantised operands (FLUX.1-schnell layer shapes)
+# ---------------------------------------------------------------------------
+GEMM_SHAPES = [(4608, 3072, 3072), (4608, 12288, 3072), (4608, 3072, 12288)]   # M, N, K
+FP4_OVER_BF16 = 4.0     # nominal dense FP4 / BF16 tensor throughput (9 / 2.25 PFLOP/s)
+
+
+def fp4_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        return bf16 * FP4_OVER_BF16, "measured bf16 burst (MEASURED_PEAKS.json) x 4, the nominal fp4/bf16 ratio"
+    except Exception:
+        return 1590.0 * FP4_OVER_BF16, "fallback bf16 1.59 PFLOP/s x 4"
+
+
+def time_gemm(kq, device, stream, K_launches: int, W: int) -> dict:
+    """kq_gemm_mxfp4 on the FLUX.1-schnell layer shapes (4608 tokens): mean
+    device time of K back-to-back launches on seeded codes and scales (the
+    cost does not depend on the values)."""
+    import torch
+    lib = kq.abi()
+    peak, src = fp4_peak()
+    out = {"kernel": "kq_gemm_mxfp4 (tcgen05 kind::mxf4 block32, fp32 out)", "peak_tflops": round(peak, 1),
+           "peak_source": src, "shapes": {}}
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    for M, N, K in GEMM_SHAPES:
+        ca = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=device, generator=g)
+        cb = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=device, generator=g)
+        ta = kq.kq_sf_tile(torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device=device, generator=g))
+        tb = kq.kq_sf_tile(torch.randint(120, 134, (N, K // 32), dtype=torch.uint8, device=device, generator=g))
+        Y = torch.empty((M, N), dtype=torch.float32, device=device)
+
+        def go():
+            st = lib.kq_gemm_mxfp4(ca.data_ptr(), ta.data_ptr(), cb.data_ptr(), tb.data_ptr(), M, N, K,
+                                   Y.data_ptr(), stream.cuda_stream)
+            if st != 0:
+                raise RuntimeError(lib.kq_last_error().decode())
+        for _ in range(W):
+            go()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K_launches):
+            go()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) / K_launches * 1e3
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        out["shapes"][f"{M}x{N}x{K}"] = {"us": round(us, 2), "tflops": round(tf, 1),
+                                         "frac_of_peak": round(tf / peak, 4)}
+        del ca, cb, ta, tb, Y
+    return out
+
+
+# ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
 def run_kroquant(args) -> int:
@@ -434,6 +491,7 @@ def run_kroquant(args) -> int:
     launch_sq = [timed_burst(i, "sq", K, W) for i in range(len(rings))]
     launch_tc = timed_burst(dominant, "tc", K, W)
     weight_side = time_weight_side(kq, device, stream, K, W)
+    w4a4_gemm = time_gemm(kq, device, stream, K, W)
 
     # end to end through the public API: pinned host input -> device -> quantize -> host.
     # PCIe is full duplex, so the device-to-host read of one launch's codes
@@ -559,6 +617,7 @@ def run_kroquant(args) -> int:
                 "frac_of_peak": round(dom_bytes / (launch_tc * 1e-3) / 1e9 / peak, 4),
             },
             "weight_side": weight_side,
+            "w4a4_gemm": w4a4_gemm,
             "e2e": {
                 "value": round(e2e_value, 2),
                 "unit": UNIT,

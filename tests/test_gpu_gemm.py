@@ -51,7 +51,7 @@ def test_sf_tile_matches_oracle(kq, R, K):
     assert np.array_equal(t, o.sf_tile(s))
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (200, 72, 384), (256, 384, 1024), (1, 1, 128)])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (200, 72, 384), (256, 384, 1024), (1, 1, 128), (300, 1029, 256)])
 def test_gemm_unit_scales_is_exact(kq, M, N, K):
     """Unit scales: every product is a multiple of 1/4 below 36 and every sum
     fits fp32 exactly, so any accumulation order gives the oracle's bits.  A

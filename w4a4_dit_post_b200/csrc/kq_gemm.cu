@@ -21,7 +21,9 @@
 // layout), one bulk copy of each 512-byte scale block, two MMAs of K = 64.
 // Roles (192 threads): warp 0 lane 0 loads (S stages), warp 1 owns tensor
 // memory and lane 0 issues the scale copies and MMAs, warps 2..5 read the
-// accumulator (one row per thread) and store fp32 rows.  Every wait is
+// accumulator (one row per thread) 32 columns at a time and stage each
+// 128 x 32 fp32 slice in shared memory (128-byte swizzle) for a TMA tensor
+// store (when N is a multiple of 4; otherwise they store rows directly).  Every wait is
 // bounded; a wait that runs out sets the device status word and the CTA
 // drains and exits.
 #include <cuda.h>
@@ -41,10 +43,12 @@ namespace gemm {
 constexpr int kThreads = 192;
 constexpr int kTile = 128;          // M and N of the CTA tile (and of the MMA)
 constexpr int kKStep = 128;         // K per stage (fp4 elements)
-constexpr int kStages = 6;
+constexpr int kStages = 5;
 constexpr int kOpBytes = kTile * kKStep / 2;        // 8 KiB of codes per operand per stage
 constexpr int kSfBytes = 512;
 constexpr int kStageBytes = 2 * kOpBytes + 2 * kSfBytes;
+constexpr int kChunkBytes = kTile * 128;           // one 128-row x 32-column fp32 slice of Y
+constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 256;      // 128 accumulator columns + 8 scale columns
 constexpr int kSfaCol = 128, kSfbCol = 132;
 
@@ -90,6 +94,34 @@ __device__ __forceinline__ void fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const void* tmap, int c0, int c1, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void epi_barrier() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+}
+// Barrier 1 among the epilogue warps that also ORs a flag across them, so
+// that all of them take the same branch (none is left at a barrier).
+__device__ __forceinline__ bool epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(kEpiThreads)
+      : "memory");
+  return r != 0;
+}
+
 // 1-D bulk copy global -> shared, completion on an mbarrier (16-byte aligned).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -117,19 +149,21 @@ struct GemmArgs {
   const uint8_t* sfa;        // blocked scales of A: [ceil(M/128)][K/128][512]
   const uint8_t* sfb;        // blocked scales of B
   float* Y;                  // [M][N] fp32
+  int tma_store;             // 1: Y leaves through shared memory and TMA stores (N % 4 == 0)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-            const GemmArgs args, unsigned int* devstat) {
+            const __grid_constant__ CUtensorMap ymap, const GemmArgs args, unsigned int* devstat) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* out_chunk = smem + kStages * kStageBytes;               // [128 rows][128 B], 128B swizzle
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_chunk + kChunkBytes);
   const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kStages]);
   const uint32_t accf = smem_addr(&bars[2 * kStages]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 1));
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 2));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kStages + 1]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kStages + 2]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_tile = blockIdx.x, m_tile = blockIdx.y;
@@ -139,6 +173,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
   if (tid == 0) {
     tma_prefetch_desc(&amap);
     tma_prefetch_desc(&bmap);
+    if (args.tma_store) tma_prefetch_desc(&ymap);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
@@ -229,28 +264,38 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
     const int q = warp & 3;
     const int row = m_tile * kTile + 32 * q + lane;
     const bool ok = mbar_wait_bounded(accf, 0);
-    if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
+    if (epi_any(!ok || *abort_flag)) {
       if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
     } else {
       fence_after_sync();
       const int n0 = n_tile * kTile;
+      const int etid = tid - 64;
+      const int r_local = 32 * q + lane;
       for (int c = 0; c < kTile / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
-        if (row < args.M) {
+        if (args.tma_store) {
+          // the previous slice's store has read the staging chunk
+          if (etid == 0) bulk_wait_read_all();
+          epi_barrier();
+          uint8_t* row = out_chunk + r_local * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(row + ((u ^ (r_local & 7)) << 4)) =
+                make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          epi_barrier();
+          if (etid == 0) {
+            tma_store_2d(&ymap, n0 + 32 * c, m_tile * kTile, smem_addr(out_chunk));
+            bulk_commit();
+          }
+        } else if (row < args.M) {
           float* dst = args.Y + (size_t)row * args.N + n0 + 32 * c;
           const int n_valid = args.N - (n0 + 32 * c);
-          if (n_valid >= 32 && (args.N & 3) == 0) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              reinterpret_cast<float4*>(dst)[i] =
-                  make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                              __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-          } else {
-            for (int i = 0; i < 32 && i < n_valid; ++i) dst[i] = __uint_as_float(r[i]);
-          }
+          for (int i = 0; i < 32 && i < n_valid; ++i) dst[i] = __uint_as_float(r[i]);
         }
       }
+      if (args.tma_store && etid == 0) bulk_wait_all();
     }
   }
 
@@ -356,7 +401,7 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return kq::cuda_fail(err, "cudaGetDevice");
   if (dev < 0 || dev >= kq::kMaxDevices) return kq::fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
-  const size_t smem = 1024 + (size_t)kq::gemm::kStages * kq::gemm::kStageBytes + 256;
+  const size_t smem = 1024 + (size_t)kq::gemm::kStages * kq::gemm::kStageBytes + kq::gemm::kChunkBytes + 256;
   static std::once_flag attr_once[kq::kMaxDevices];
   static cudaError_t attr_err[kq::kMaxDevices];
   std::call_once(attr_once[dev], [&] {
@@ -365,9 +410,23 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   });
   if (attr_err[dev] != cudaSuccess) return kq::cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
 
-  CUtensorMap am, bm;
+  CUtensorMap am, bm, ym;
   if (int st = kq::codes_tmap(&am, a_codes, M, K)) return st;
   if (int st = kq::codes_tmap(&bm, b_codes, N, K)) return st;
+  const bool tma_store = (N % 4) == 0;
+  memset(&ym, 0, sizeof(ym));
+  if (tma_store) {
+    // Y [M][N] fp32; box 32 columns (128 bytes) x 128 rows, 128-byte swizzle
+    PFN_cuTensorMapEncodeTiled_v12000 enc = kq::gemm_encoder();
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+    const cuuint32_t box[2] = {32, (cuuint32_t)kq::gemm::kTile};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(&ym, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Y, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return kq::fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed (CUresult %d)", (int)r);
+  }
   kq::gemm::GemmArgs args;
   args.M = (int)M;
   args.N = (int)N;
@@ -376,6 +435,7 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   args.sfa = a_sf_tiled;
   args.sfb = b_sf_tiled;
   args.Y = Y;
+  args.tma_store = tma_store ? 1 : 0;
   unsigned int* devstat = nullptr;
   if (int st = kq::device_status_address(&devstat)) return st;
 
@@ -389,7 +449,7 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel, am, bm, args, devstat);
+  err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel, am, bm, ym, args, devstat);
   if (err != cudaSuccess) return kq::cuda_fail(err, "gemm_kernel launch");
   return kq::check_launch("gemm_kernel launch");
 }
