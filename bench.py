@@ -305,7 +305,7 @@ def fp4_peak():
         return 1590.0 * FP4_OVER_BF16, "fallback bf16 1.59 PFLOP/s x 4"
 
 
-def time_gemm(kq, device, stream, K_launches: int, W: int) -> dict:
+def time_gemm(kq, device, stream, K_launches: int, W: int, shapes=None) -> dict:
     """kq_gemm_mxfp4 on the FLUX.1-schnell layer shapes (4608 tokens): mean
     device time of K back-to-back launches on seeded codes and scales (the
     cost does not depend on the values)."""
@@ -316,7 +316,7 @@ def time_gemm(kq, device, stream, K_launches: int, W: int) -> dict:
            "peak_source": src, "shapes": {}}
     g = torch.Generator(device=device)
     g.manual_seed(7)
-    for M, N, K in GEMM_SHAPES:
+    for M, N, K in (shapes or GEMM_SHAPES):
         ca = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=device, generator=g)
         cb = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=device, generator=g)
         ta = kq.kq_sf_tile(torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device=device, generator=g))
@@ -451,6 +451,15 @@ def run_kroquant(args) -> int:
         return e0.elapsed_time(e1) / K
 
     K, W = args.steps, args.warmup
+    if args.profile == "gemm":
+        # only kq_gemm_mxfp4 launches on the first FLUX layer shape (for ncu captures)
+        M, N, Kd = GEMM_SHAPES[0]
+        r = time_gemm(kq, device, stream, K, W, shapes=[GEMM_SHAPES[0]])
+        if rank == 0:
+            print(json.dumps({"profile": f"kq_gemm_mxfp4 {M}x{N}x{Kd}", "launches": W + K,
+                              **r["shapes"][f"{M}x{N}x{Kd}"],
+                              "device_status": kq.kq_device_status(device)}), flush=True)
+        return 0
     if args.profile:
         # only the launches of one kernel on the largest shape (for ncu captures)
         fn = "tc" if args.profile == "tc" else "kq"
@@ -723,9 +732,10 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["kroquant", "reference"], default="kroquant")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", nargs="?", const="kq", choices=["kq", "tc"], default=None,
-                    help="run only the kq_quantize (or kq_quantize_tc) launches of the largest "
-                         "shape, for ncu captures")
+    ap.add_argument("--profile", nargs="?", const="kq", choices=["kq", "tc", "gemm"], default=None,
+                    help="run only the kq_quantize (kq), kq_quantize_tc (tc) launches of the largest "
+                         "shape, or the kq_gemm_mxfp4 launches of the first layer shape (gemm), "
+                         "for ncu captures")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     _, world, _ = dist_env()
