@@ -218,18 +218,19 @@ def hbm_peak():
 
 def ncu_traffic():
     """DRAM bytes per launch of the d=12288 kq_quantize launch from the
-    committed ncu summary, if it was taken on the current sources."""
+    committed ncu summary, if it was taken on the current sources of the
+    streaming kernel."""
     path = os.path.join(ROOT, "profiles", "kq_quantize_flux.md")
     try:
         from w4a4_dit_post_b200 import build
-        cur = build.source_hash()
+        cur = build.stream_kernel_hash()
         vals = {}
         with open(path) as f:
             for line in f:
                 if line.startswith("<!-- ") and "=" in line:
                     k, v = line[5:].split("-->")[0].strip().split("=", 1)
                     vals[k.strip()] = v.strip()
-        if vals.get("source_hash") == cur and "traffic_bytes_per_launch" in vals:
+        if vals.get("stream_kernel_hash") == cur and "traffic_bytes_per_launch" in vals:
             return float(vals["traffic_bytes_per_launch"]), "ncu (current sources)"
         return None, "ncu summary predates the current kernel sources"
     except Exception as e:

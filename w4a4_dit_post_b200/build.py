@@ -65,6 +65,23 @@ def source_hash() -> str:
     return _hash_inputs()
 
 
+# the translation unit of the streaming kernels and everything it includes
+STREAM_KERNEL_FILES = ("csrc/kq_stream.cu", "csrc/kq_device.cuh", "csrc/kq_host.h", "../include/kq.h")
+
+
+def stream_kernel_hash() -> str:
+    """Hash of the sources the streaming kernels (kq_quantize, sq_quantize,
+    kq_transform) are compiled from, and of the compile flags."""
+    h = hashlib.sha256()
+    h.update(" ".join(ARCH_FLAGS).encode())
+    for rel in STREAM_KERNEL_FILES:
+        path = os.path.normpath(os.path.join(os.path.dirname(os.path.abspath(__file__)), rel))
+        h.update(rel.encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def is_current() -> bool:
     if not os.path.exists(LIB_PATH) or not os.path.exists(HASH_PATH):
         return False
