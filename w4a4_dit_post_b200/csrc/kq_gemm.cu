@@ -15,7 +15,8 @@
 // bytes, copied into all four lane quarters).  kq_sf_tile rewrites the
 // row-major scale bytes into such 512-byte blocks once per operand.
 //
-// Tiling.  One CTA computes a 128 x 128 tile of Y; K advances in steps of 128
+// Tiling.  Y is cut into 128 x 128 tiles; persistent CTAs (two per SM) walk
+// them.  Within a tile K advances in steps of 128
 // (64 bytes of codes per row, 4 scales): per step one TMA load of A and of B
 // (128 rows x 64 bytes, 64-byte swizzle: the canonical K-major operand
 // layout), one bulk copy of each 512-byte scale block, two MMAs of K = 64.
@@ -148,10 +149,20 @@ struct GemmArgs {
   int k_steps;               // K / 128
   const uint8_t* sfa;        // blocked scales of A: [ceil(M/128)][K/128][512]
   const uint8_t* sfb;        // blocked scales of B
+  int m_tiles, n_tiles;
   float* Y;                  // [M][N] fp32
   int tma_store;             // 1: Y leaves through shared memory and TMA stores (N % 4 == 0)
 };
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Persistent: CTA b takes tiles b, b + G, b + 2G, ... (tile t = (t % m_tiles,
+// t / m_tiles), so CTAs running together share B tiles in L2).  The stage
+// ring runs on across tiles, and the accumulator is handed back to the MMA
+// lane as soon as the epilogue has read it, so the next tile's loads and MMAs
+// overlap this tile's stores; two CTAs share an SM.
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
             const __grid_constant__ CUtensorMap ymap, const GemmArgs args, unsigned int* devstat) {
@@ -161,13 +172,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
   uint8_t* out_chunk = smem + kStages * kStageBytes;               // [128 rows][128 B], 128B swizzle
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_chunk + kChunkBytes);
   const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kStages]);
-  const uint32_t accf = smem_addr(&bars[2 * kStages]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kStages + 1]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kStages + 2]);
+  const uint32_t accf = smem_addr(&bars[2 * kStages]), acce = smem_addr(&bars[2 * kStages + 1]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kStages + 2]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kStages + 3]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_tile = blockIdx.x, m_tile = blockIdx.y;
   const int KS = args.k_steps;
+  const int n_tiles_total = args.m_tiles * args.n_tiles;
+  const int my_tiles = (int)blockIdx.x < n_tiles_total
+                           ? (n_tiles_total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                           : 0;
 
   pdl_launch_dependents();
   if (tid == 0) {
@@ -179,6 +193,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init(accf, 1);
+    mbar_init(acce, kEpiThreads / 32);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -197,91 +212,114 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint8_t* sfa_tile = args.sfa + (size_t)m_tile * KS * kSfBytes;
-      const uint8_t* sfb_tile = args.sfb + (size_t)n_tile * KS * kSfBytes;
-      int issued = 0;
-      for (int kt = 0; kt < KS; ++kt) {
-        const int s = kt % kStages;
-        if (kt >= kStages && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(kt / kStages - 1) & 1u)) {
-          *abort_flag = 1;
-          atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
-          break;
+      int issued = 0, seq = 0;
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
+        const uint8_t* sfa_tile = args.sfa + (size_t)m_tile * KS * kSfBytes;
+        const uint8_t* sfb_tile = args.sfb + (size_t)n_tile * KS * kSfBytes;
+        for (int kt = 0; kt < KS; ++kt, ++seq) {
+          const int s = seq % kStages;
+          if (seq >= kStages && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(seq / kStages - 1) & 1u)) {
+            *abort_flag = 1;
+            atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+            break;
+          }
+          if (*abort_flag) break;
+          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t bar = full0 + 8 * s;
+          mbar_arrive_expect_tx(bar, (uint32_t)kStageBytes);
+          tma_load_2d(smem_addr(st), &amap, kt * (kKStep / 2), m_tile * kTile, bar);
+          tma_load_2d(smem_addr(st + kOpBytes), &bmap, kt * (kKStep / 2), n_tile * kTile, bar);
+          bulk_load(smem_addr(st + 2 * kOpBytes), sfa_tile + (size_t)kt * kSfBytes, kSfBytes, bar);
+          bulk_load(smem_addr(st + 2 * kOpBytes + kSfBytes), sfb_tile + (size_t)kt * kSfBytes, kSfBytes, bar);
+          issued = seq + 1;
         }
-        if (*abort_flag) break;
-        uint8_t* st = smem + s * kStageBytes;
-        const uint32_t bar = full0 + 8 * s;
-        mbar_arrive_expect_tx(bar, (uint32_t)kStageBytes);
-        tma_load_2d(smem_addr(st), &amap, kt * (kKStep / 2), m_tile * kTile, bar);
-        tma_load_2d(smem_addr(st + kOpBytes), &bmap, kt * (kKStep / 2), n_tile * kTile, bar);
-        bulk_load(smem_addr(st + 2 * kOpBytes), sfa_tile + (size_t)kt * kSfBytes, kSfBytes, bar);
-        bulk_load(smem_addr(st + 2 * kOpBytes + kSfBytes), sfb_tile + (size_t)kt * kSfBytes, kSfBytes, bar);
-        issued = kt + 1;
       }
       if (*abort_flag) {
         const int lo = issued > kStages ? issued - kStages : 0;
-        for (int kt = lo; kt < issued; ++kt)
-          (void)mbar_wait_bounded(full0 + 8 * (kt % kStages), (uint32_t)(kt / kStages) & 1u);
+        for (int q = lo; q < issued; ++q)
+          (void)mbar_wait_bounded(full0 + 8 * (q % kStages), (uint32_t)(q / kStages) & 1u);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      int seq = 0;
       bool issued_any = false;
-      for (int kt = 0; kt < KS; ++kt) {
-        const int s = kt % kStages;
-        if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)(kt / kStages) & 1u) || *abort_flag) {
+      for (int i = 0; i < my_tiles; ++i) {
+        // the epilogue has read the previous tile's accumulator
+        bool ok = i == 0 || mbar_wait_bounded(acce, (uint32_t)(i - 1) & 1u);
+        if (ok) fence_after_sync();
+        for (int kt = 0; ok && kt < KS; ++kt, ++seq) {
+          const int s = seq % kStages;
+          ok = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(seq / kStages) & 1u) && !*abort_flag;
+          if (!ok) break;
+          fence_after_sync();
+          const uint32_t st = smem_addr(smem + s * kStageBytes);
+          // scale blocks of this step into tensor memory (in issue order with
+          // the MMAs below, and after the MMAs of the previous step)
+          sf_copy(tmem_base + kSfaCol, sf_desc(st + 2 * kOpBytes));
+          sf_copy(tmem_base + kSfbCol, sf_desc(st + 2 * kOpBytes + kSfBytes));
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint32_t sf_id = (uint32_t)(2 * kk);      // scales 2kk, 2kk+1 of the group of 4
+            const uint32_t sfa = (tmem_base + kSfaCol) | (sf_id << 30);
+            const uint32_t sfb = (tmem_base + kSfbCol) | (sf_id << 30);
+            const uint32_t idesc = kIdescBase | (sf_id << 29) | (sf_id << 4);
+            mma_mxf4(tmem_base, sw64_desc(st + kk * 32), sw64_desc(st + kOpBytes + kk * 32), idesc,
+                     sfa, sfb, (kt | kk) != 0);
+          }
+          mma_commit(empty0 + 8 * s);
+          issued_any = true;
+        }
+        if (!ok) {
           *abort_flag = 1;
           atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
           break;
         }
-        fence_after_sync();
-        const uint32_t st = smem_addr(smem + s * kStageBytes);
-        // scale blocks of this step into tensor memory (in issue order with
-        // the MMAs below, and after the MMAs of the previous step)
-        sf_copy(tmem_base + kSfaCol, sf_desc(st + 2 * kOpBytes));
-        sf_copy(tmem_base + kSfbCol, sf_desc(st + 2 * kOpBytes + kSfBytes));
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint32_t sf_id = (uint32_t)(2 * kk);      // scales 2kk, 2kk+1 of the group of 4
-          const uint32_t sfa = (tmem_base + kSfaCol) | (sf_id << 30);
-          const uint32_t sfb = (tmem_base + kSfbCol) | (sf_id << 30);
-          const uint32_t idesc = kIdescBase | (sf_id << 29) | (sf_id << 4);
-          mma_mxf4(tmem_base, sw64_desc(st + kk * 32), sw64_desc(st + kOpBytes + kk * 32), idesc,
-                   sfa, sfb, (kt | kk) != 0);
-        }
-        mma_commit(empty0 + 8 * s);
-        issued_any = true;
+        mma_commit(accf);
       }
-      if (!*abort_flag) {
-        mma_commit(accf);
-      } else if (issued_any) {
-        // let the MMAs already issued finish before tensor memory is freed
-        mma_commit(accf);
-        (void)mbar_wait_bounded(accf, 0);
+      if (*abort_flag && issued_any) {
+        // give the MMAs already issued (microseconds of work) time to finish
+        // before tensor memory is freed
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 20000000ull) {}
       }
     }
   } else {
-    // epilogue: warps 2..5 -> TMEM lane quarters (warp % 4)
+    // epilogue: warps 2..5 -> TMEM lane quarters (warp % 4); thread = one row
     const int q = warp & 3;
-    const int row = m_tile * kTile + 32 * q + lane;
-    const bool ok = mbar_wait_bounded(accf, 0);
-    if (epi_any(!ok || *abort_flag)) {
-      if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
-    } else {
+    const int etid = tid - 64;
+    const int r_local = 32 * q + lane;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int t = (int)blockIdx.x + i * (int)gridDim.x;
+      const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
+      const int row = m_tile * kTile + r_local;
+      const bool ok = mbar_wait_bounded(accf, (uint32_t)i & 1u);
+      if (epi_any(!ok || *abort_flag)) {
+        if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
       fence_after_sync();
       const int n0 = n_tile * kTile;
-      const int etid = tid - 64;
-      const int r_local = 32 * q + lane;
       for (int c = 0; c < kTile / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+        if (c == kTile / 32 - 1) {
+          // the whole accumulator is in registers or staged: hand it back
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acce);
+        }
         if (args.tma_store) {
           // the previous slice's store has read the staging chunk
           if (etid == 0) bulk_wait_read_all();
           epi_barrier();
-          uint8_t* row = out_chunk + r_local * 128;
+          uint8_t* rowp = out_chunk + r_local * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(row + ((u ^ (r_local & 7)) << 4)) =
+            *reinterpret_cast<uint4*>(rowp + ((u ^ (r_local & 7)) << 4)) =
                 make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           epi_barrier();
@@ -292,11 +330,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
         } else if (row < args.M) {
           float* dst = args.Y + (size_t)row * args.N + n0 + 32 * c;
           const int n_valid = args.N - (n0 + 32 * c);
-          for (int i = 0; i < 32 && i < n_valid; ++i) dst[i] = __uint_as_float(r[i]);
+          for (int k = 0; k < 32 && k < n_valid; ++k) dst[k] = __uint_as_float(r[k]);
         }
       }
-      if (args.tma_store && etid == 0) bulk_wait_all();
     }
+    if (args.tma_store && etid == 0) bulk_wait_all();
   }
 
   fence_before_sync();
@@ -393,8 +431,8 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   if (!kq::aligned(a_codes, 16) || !kq::aligned(b_codes, 16) || !kq::aligned(a_sf_tiled, 16) ||
       !kq::aligned(b_sf_tiled, 16) || !kq::aligned(Y, 16))
     return kq::fail(KQ_ERR_ALIGNMENT, "%s: codes, tiled scales and Y must be 16-byte aligned", fn);
-  if ((M + 127) / 128 > 65535 || N >= ((int64_t)1 << 31) / 128 || K >= ((int64_t)1 << 24) ||
-      M * N >= ((int64_t)1 << 40))
+  if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 24) ||
+      ((M + 127) / 128) * ((N + 127) / 128) >= ((int64_t)1 << 31))
     return kq::fail(KQ_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", fn);
 
   int dev = 0;
@@ -436,11 +474,17 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   args.sfb = b_sf_tiled;
   args.Y = Y;
   args.tma_store = tma_store ? 1 : 0;
+  args.m_tiles = (int)((M + 127) / 128);
+  args.n_tiles = (int)((N + 127) / 128);
   unsigned int* devstat = nullptr;
   if (int st = kq::device_status_address(&devstat)) return st;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((N + 127) / 128), (unsigned)((M + 127) / 128));
+  int sms = 0;
+  if (int st = kq::sm_count(&sms)) return st;
+  const int64_t tiles = (int64_t)args.m_tiles * args.n_tiles;
+  const int64_t slots = 2 * (int64_t)sms;                    // two CTAs per SM
+  cfg.gridDim = dim3((unsigned)(tiles < slots ? tiles : slots));
   cfg.blockDim = dim3(kq::gemm::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = kq::as_stream(stream);
