@@ -347,6 +347,62 @@ def time_gemm(kq, device, stream, K_launches: int, W: int, shapes=None) -> dict:
     return out
 
 
+def time_layer(kq, device, stream, K_launches: int, W: int) -> dict:
+    """One W4A4 linear layer per FLUX.1-schnell layer shape, per step:
+    kq_quantize on the bf16 activations, kq_sf_tile on their scales and
+    kq_gemm_mxfp4 against weights quantised offline (kq_quantize_weights),
+    against the same layer as a bf16 GEMM (torch.matmul, cuBLAS) on the
+    unquantised operands.  Mean device time of K back-to-back steps."""
+    import torch
+    lib = kq.abi()
+    out = {"step": "kq_quantize + kq_sf_tile + kq_gemm_mxfp4 (weights quantised offline)",
+           "baseline": "torch.matmul bf16 (cuBLAS), same X and W", "shapes": {}}
+    for M, N, K in GEMM_SHAPES:
+        wd = synthetic.Workload("layer", M, K, "bf16", "normal", 0.01, None, 100.0, 4.0, 3)
+        raw = synthetic.make_activations(wd)
+        x = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16).to(device)
+        p = torch.from_numpy(synthetic.make_params(K // 32, 3)).to(device)
+        Wt = torch.from_numpy(synthetic.make_weights(N, K, 31)).to(device)
+        cw, sw = kq.kq_quantize_weights(Wt, p)
+        tw = kq.kq_sf_tile(sw)
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty((M, K // 32), dtype=torch.uint8, device=device)
+        tiled = torch.empty(((M + 127) // 128, K // 128, 512), dtype=torch.uint8, device=device)
+        Y = torch.empty((M, N), dtype=torch.float32, device=device)
+        Wb = Wt.to(torch.bfloat16)
+        s = stream.cuda_stream
+
+        def step():
+            st = lib.kq_quantize(x.data_ptr(), kq.KQ_DTYPE_BF16, M, K, p.data_ptr(), codes.data_ptr(),
+                                 scales.data_ptr(), s)
+            st = st or lib.kq_sf_tile(scales.data_ptr(), M, K, tiled.data_ptr(), s)
+            st = st or lib.kq_gemm_mxfp4(codes.data_ptr(), tiled.data_ptr(), cw.data_ptr(), tw.data_ptr(),
+                                         M, N, K, Y.data_ptr(), s)
+            if st != 0:
+                raise RuntimeError(lib.kq_last_error().decode())
+
+        def base():
+            torch.matmul(x, Wb.t())
+
+        res = {}
+        for name, fn in (("w4a4", step), ("bf16", base)):
+            for _ in range(W):
+                fn()
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(K_launches):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            res[name] = e0.elapsed_time(e1) / K_launches * 1e3
+        out["shapes"][f"{M}x{N}x{K}"] = {"w4a4_us": round(res["w4a4"], 2), "bf16_us": round(res["bf16"], 2),
+                                         "speedup": round(res["bf16"] / res["w4a4"], 3)}
+        del x, p, Wt, cw, sw, tw, codes, scales, tiled, Y, Wb
+    return out
+
+
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
@@ -502,6 +558,7 @@ def run_kroquant(args) -> int:
     launch_tc = timed_burst(dominant, "tc", K, W)
     weight_side = time_weight_side(kq, device, stream, K, W)
     w4a4_gemm = time_gemm(kq, device, stream, K, W)
+    w4a4_layer = time_layer(kq, device, stream, K, W)
 
     # end to end through the public API: pinned host input -> device -> quantize -> host.
     # PCIe is full duplex, so the device-to-host read of one launch's codes
@@ -628,6 +685,7 @@ def run_kroquant(args) -> int:
             },
             "weight_side": weight_side,
             "w4a4_gemm": w4a4_gemm,
+            "w4a4_layer": w4a4_layer,
             "e2e": {
                 "value": round(e2e_value, 2),
                 "unit": UNIT,

@@ -181,7 +181,7 @@ int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void
  *   folded weights (codes [N][K/2] from kq_quantize_weights, scales tiled).
  *   Y [M][N] fp32 row-major.  Products on the tensor cores with the
  *   block-scaled FP4 MMA, fp32 accumulation in tensor memory.
- *   K a multiple of 128; all pointers 16-byte aligned; ceil(M/128) <= 65535.
+ *   K a multiple of 128; all pointers 16-byte aligned; M, N < 2^31.
  */
 int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
                   const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, float* Y,

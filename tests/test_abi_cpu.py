@@ -116,7 +116,7 @@ def test_other_argument_checks(lib):
     assert g(A16 + 8, A16b, A16c, A16d, 128, 128, 256, A16, None) == 2
     assert g(A16, A16b, A16c, A16d, 0, 128, 256, None, None) == 0
     assert g(A16, A16b, None, A16d, 128, 128, 256, A16, None) == 1
-    assert g(A16, A16b, A16c, A16d, 65536 * 128, 128, 256, A16, None) == 4
+    assert g(A16, A16b, A16c, A16d, 2 ** 31, 128, 256, A16, None) == 4
     assert lib.kq_dequant(A16, A16b, 4, 64, A16c + 4, None) == 2
     assert lib.kq_dequant(A16, A16b, 0, 64, A16c, None) == 0
     assert lib.kq_device_status(None, 0) == 1
