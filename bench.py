@@ -349,13 +349,14 @@ def time_gemm(kq, device, stream, K_launches: int, W: int, shapes=None) -> dict:
 
 def time_layer(kq, device, stream, K_launches: int, W: int) -> dict:
     """One W4A4 linear layer per FLUX.1-schnell layer shape, per step:
-    kq_quantize on the bf16 activations, kq_sf_tile on their scales and
-    kq_gemm_mxfp4 against weights quantised offline (kq_quantize_weights),
+    kq_quantize_sf_tiled on the bf16 activations (codes, and scales in the
+    GEMM's block layout) and kq_gemm_mxfp4 against weights quantised offline
+    (kq_quantize_weights),
     against the same layer as a bf16 GEMM (torch.matmul, cuBLAS) on the
     unquantised operands.  Mean device time of K back-to-back steps."""
     import torch
     lib = kq.abi()
-    out = {"step": "kq_quantize + kq_sf_tile + kq_gemm_mxfp4 (weights quantised offline)",
+    out = {"step": "kq_quantize_sf_tiled + kq_gemm_mxfp4 (weights quantised offline)",
            "baseline": "torch.matmul bf16 (cuBLAS), same X and W", "shapes": {}}
     for M, N, K in GEMM_SHAPES:
         wd = synthetic.Workload("layer", M, K, "bf16", "normal", 0.01, None, 100.0, 4.0, 3)
@@ -366,16 +367,14 @@ def time_layer(kq, device, stream, K_launches: int, W: int) -> dict:
         cw, sw = kq.kq_quantize_weights(Wt, p)
         tw = kq.kq_sf_tile(sw)
         codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
-        scales = torch.empty((M, K // 32), dtype=torch.uint8, device=device)
         tiled = torch.empty(((M + 127) // 128, K // 128, 512), dtype=torch.uint8, device=device)
         Y = torch.empty((M, N), dtype=torch.float32, device=device)
         Wb = Wt.to(torch.bfloat16)
         s = stream.cuda_stream
 
         def step():
-            st = lib.kq_quantize(x.data_ptr(), kq.KQ_DTYPE_BF16, M, K, p.data_ptr(), codes.data_ptr(),
-                                 scales.data_ptr(), s)
-            st = st or lib.kq_sf_tile(scales.data_ptr(), M, K, tiled.data_ptr(), s)
+            st = lib.kq_quantize_sf_tiled(x.data_ptr(), kq.KQ_DTYPE_BF16, M, K, p.data_ptr(),
+                                          codes.data_ptr(), tiled.data_ptr(), s)
             st = st or lib.kq_gemm_mxfp4(codes.data_ptr(), tiled.data_ptr(), cw.data_ptr(), tw.data_ptr(),
                                          M, N, K, Y.data_ptr(), s)
             if st != 0:
@@ -399,7 +398,7 @@ def time_layer(kq, device, stream, K_launches: int, W: int) -> dict:
             res[name] = e0.elapsed_time(e1) / K_launches * 1e3
         out["shapes"][f"{M}x{N}x{K}"] = {"w4a4_us": round(res["w4a4"], 2), "bf16_us": round(res["bf16"], 2),
                                          "speedup": round(res["bf16"] / res["w4a4"], 3)}
-        del x, p, Wt, cw, sw, tw, codes, scales, tiled, Y, Wb
+        del x, p, Wt, cw, sw, tw, codes, tiled, Y, Wb
     return out
 
 

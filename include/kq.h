@@ -108,6 +108,17 @@ int kq_quantize_tc(const void* x, int x_dtype, int64_t M, int64_t d,
                    void* stream);
 
 /*
+ * kq_quantize_sf_tiled -- kq_quantize with the scale bytes written straight
+ * into the blocked layout of kq_sf_tile (the operand format of
+ * kq_gemm_mxfp4), saving that pass in a layer step; codes as kq_quantize.
+ *   scales_tiled [ceil(M/128)][d/128][512] uint8; its bytes for rows past M
+ *   are not written.  d a multiple of 128; other arguments as kq_quantize.
+ */
+int kq_quantize_sf_tiled(const void* x, int x_dtype, int64_t M, int64_t d,
+                         const float* params, uint8_t* codes, uint8_t* scales_tiled,
+                         void* stream);
+
+/*
  * kq_transform -- the transform stage alone: y = blockdiag(T_j) x in fp32.
  * Same arguments and limits as kq_quantize; y [M][d] fp32, 16-byte aligned.
  * It runs the same transform code as kq_quantize, so kq_quantize's codes are

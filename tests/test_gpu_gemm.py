@@ -90,3 +90,20 @@ def test_gemm_on_quantized_layer(kq):
     ref = o.gemm_mxfp4(ca, sa, cb, sb)
     tol = (w.d / 64 + 64) * 2.0 ** -23 * o.gemm_error_scale(ca, sa, cb, sb)
     assert np.all(np.abs(Y - ref) <= tol)
+
+
+@pytest.mark.parametrize("M,d", [(1, 128), (200, 1152), (4608, 3072)])
+def test_quantize_with_tiled_scales(kq, M, d):
+    """kq_quantize_sf_tiled writes the codes of kq_quantize and the scale
+    blocks kq_sf_tile makes from kq_quantize's scales (rows past M untouched)."""
+    w = synthetic.Workload("sft", M, d, "bf16", "normal", 0.01, None, 50.0, 2.0, 23)
+    raw = synthetic.make_activations(w)
+    x = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16).cuda()
+    p = torch.from_numpy(synthetic.make_params(w.nb, 23)).cuda()
+    c1, s1 = kq.kq_quantize(x, p)
+    t1 = kq.kq_sf_tile(s1)
+    c2 = torch.empty_like(c1)
+    t2 = torch.zeros_like(t1)
+    kq.kq_quantize_sf_tiled(x, p, c2, t2)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2) and torch.equal(t1, t2)

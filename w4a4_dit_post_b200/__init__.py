@@ -19,7 +19,7 @@ import torch
 from .build import LIB_PATH
 
 __all__ = [
-    "abi", "kq_quantize", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
+    "abi", "kq_quantize", "kq_quantize_sf_tiled", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
     "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4", "kq_dequant",
     "kq_device_status",
     "kq_selftest_bounded_wait",
@@ -43,6 +43,8 @@ _int = ctypes.c_int
 _SIGNATURES = {
     "kq_quantize": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_quantize_tc": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "kq_quantize_sf_tiled": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p,
+                                    _c_void_p]),
     "kq_transform": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
     "sq_quantize": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_expand_params": (_int, [_c_void_p, _i64, _c_void_p, _c_void_p]),
@@ -144,6 +146,22 @@ def kq_quantize(x, params, codes=None, scales=None):
             x.data_ptr(), _x_dtype(x), M, d, params.data_ptr(), codes.data_ptr(),
             scales.data_ptr(), _stream(x)))
     return codes, scales
+
+
+def kq_quantize_sf_tiled(x, params, codes=None, scales_tiled=None):
+    """kq_quantize with the scales in the blocked layout kq_gemm_mxfp4 reads:
+    (codes uint8 [M, d/2], scales_tiled uint8 [ceil(M/128), d/128, 512])."""
+    _need_cuda("x", x, _ACT, 2)
+    _need_cuda("params", params, (torch.float32,))
+    M, d = x.shape
+    codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
+    scales_tiled = _out(scales_tiled, ((M + 127) // 128, d // 128 if d % 128 == 0 else 0, 512),
+                        torch.uint8, x, "scales_tiled")
+    with torch.cuda.device(x.device):
+        _check("kq_quantize_sf_tiled", abi().kq_quantize_sf_tiled(
+            x.data_ptr(), _x_dtype(x), M, d, params.data_ptr(), codes.data_ptr(),
+            scales_tiled.data_ptr(), _stream(x)))
+    return codes, scales_tiled
 
 
 def kq_quantize_tc(x, params, codes=None, scales=None):

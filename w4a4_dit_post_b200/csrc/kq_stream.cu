@@ -62,7 +62,15 @@ struct Geometry {
   int M;            // rows
   int n_row_tiles;
   int stage_bytes;  // R * C * block bytes, rounded up to 1024
+  int sf_tiled;     // 1: scale bytes in the 512-byte blocks kq_gemm_mxfp4 reads
 };
+
+// Byte of (row r, scale column s) in the blocked scale layout (512-byte block
+// per 128 rows x 4 scale columns; row r's 4 scales at (r % 32) * 16 + (r / 32 % 4) * 4).
+__device__ __forceinline__ size_t sf_tiled_offset(int r, int s, int nb) {
+  return ((size_t)(r >> 7) * (size_t)(nb >> 2) + (size_t)(s >> 2)) * 512 + (size_t)((r & 31) << 4) +
+         (size_t)(((r >> 5) & 3) << 2) + (size_t)(s & 3);
+}
 
 template <int kInBytes>
 struct InLayout;
@@ -401,11 +409,14 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], sc);
       *reinterpret_cast<uint4*>(codes + g0 * 16) = lane_codes<0>(v);
-      scales[g0] = (uint8_t)e0;
-      if (second) {
-        *reinterpret_cast<uint4*>(codes + (g0 + nb) * 16) = lane_codes<1>(v);
-        scales[g0 + nb] = (uint8_t)e1;
+      if (geo.sf_tiled) {
+        scales[sf_tiled_offset(r0, j0 + c, nb)] = (uint8_t)e0;
+        if (second) scales[sf_tiled_offset(r0 + 1, j0 + c, nb)] = (uint8_t)e1;
+      } else {
+        scales[g0] = (uint8_t)e0;
+        if (second) scales[g0 + nb] = (uint8_t)e1;
       }
+      if (second) *reinterpret_cast<uint4*>(codes + (g0 + nb) * 16) = lane_codes<1>(v);
     }
   }
 }
@@ -470,9 +481,10 @@ constexpr int kMaxDevices = 64;
 
 template <int kInBytes, Op kOp>
 int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_t* codes,
-                  uint8_t* scales, float* y, cudaStream_t stream) {
+                  uint8_t* scales, float* y, cudaStream_t stream, bool sf_tiled) {
   const int nb = (int)(d / 32);
-  const Geometry geo = make_geometry<kInBytes>(M, nb);
+  Geometry geo = make_geometry<kInBytes>(M, nb);
+  geo.sf_tiled = sf_tiled ? 1 : 0;
   auto kern = stream_kernel<kInBytes, kOp>;
   const size_t smem = smem_bytes<kInBytes, kOp>(geo);
 
@@ -524,8 +536,11 @@ int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_
 
 template <Op kOp>
 int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef,
-             uint8_t* codes, uint8_t* scales, float* y, void* stream, const char* fn) {
+             uint8_t* codes, uint8_t* scales, float* y, void* stream, const char* fn,
+             bool sf_tiled = false) {
   if (int st = check_shape(M, d, KQ_MAX_D, fn)) return st;
+  if (sf_tiled && d % 128 != 0)
+    return fail(KQ_ERR_INVALID_ARG, "%s: d must be a multiple of 128 (d = %lld)", fn, (long long)d);
   if (x_dtype != KQ_DTYPE_BF16 && x_dtype != KQ_DTYPE_F32)
     return fail(KQ_ERR_DTYPE, "%s: x_dtype = %d", fn, x_dtype);
   if (M == 0) return KQ_OK;   // nothing to read or write; pointers may be NULL
@@ -540,8 +555,8 @@ int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef
   if (codes && !aligned(codes, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: codes must be 16-byte aligned", fn);
   if (y && !aligned(y, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: y must be 16-byte aligned", fn);
   const cudaStream_t s = as_stream(stream);
-  if (x_dtype == KQ_DTYPE_BF16) return launch_stream<2, kOp>(x, M, d, coef, codes, scales, y, s);
-  return launch_stream<4, kOp>(x, M, d, coef, codes, scales, y, s);
+  if (x_dtype == KQ_DTYPE_BF16) return launch_stream<2, kOp>(x, M, d, coef, codes, scales, y, s, sf_tiled);
+  return launch_stream<4, kOp>(x, M, d, coef, codes, scales, y, s, sf_tiled);
 }
 
 }  // namespace
@@ -575,6 +590,12 @@ int kq_quantize(const void* x, int x_dtype, int64_t M, int64_t d, const float* p
                 uint8_t* codes, uint8_t* scales, void* stream) {
   return kq::dispatch<kq::Op::kKqQuant>(x, x_dtype, M, d, params, codes, scales, nullptr, stream,
                                         "kq_quantize");
+}
+
+int kq_quantize_sf_tiled(const void* x, int x_dtype, int64_t M, int64_t d, const float* params,
+                         uint8_t* codes, uint8_t* scales_tiled, void* stream) {
+  return kq::dispatch<kq::Op::kKqQuant>(x, x_dtype, M, d, params, codes, scales_tiled, nullptr,
+                                        stream, "kq_quantize_sf_tiled", true);
 }
 
 int kq_transform(const void* x, int x_dtype, int64_t M, int64_t d, const float* params, float* y,
