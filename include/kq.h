@@ -119,6 +119,27 @@ int kq_quantize_sf_tiled(const void* x, int x_dtype, int64_t M, int64_t d,
                          void* stream);
 
 /*
+ * kq_quantize_centered -- the centring variant (a per-token-mean variant of
+ * the online quantizer on the pages, from a different method): each token is
+ * shifted by its own offset before the transform, MXFP4(T (x - mu 1)); the
+ * GEMM restores the offset in full precision (kq_gemm_mxfp4_rank1).
+ *   mu [M] fp32 (4-byte aligned), normally the per-token mean (kq_row_sum
+ *   with scale 1/d); x - mu is formed in fp32.  Other arguments as kq_quantize.
+ */
+int kq_quantize_centered(const void* x, int x_dtype, int64_t M, int64_t d,
+                         const float* params, const float* mu, uint8_t* codes,
+                         uint8_t* scales, void* stream);
+
+/*
+ * kq_row_sum -- out[m] = scale * sum_k x[m][k], fp32 accumulation: the
+ * per-token means of the centring variant (scale = 1/d) and the row sums W 1
+ * of the weights its GEMM needs (scale = 1).
+ *   x [M][d] bf16 or fp32 (16-byte aligned), out [M] fp32 (4-byte aligned).
+ */
+int kq_row_sum(const void* x, int x_dtype, int64_t M, int64_t d, float scale, float* out,
+               void* stream);
+
+/*
  * kq_transform -- the transform stage alone: y = blockdiag(T_j) x in fp32.
  * Same arguments and limits as kq_quantize; y [M][d] fp32, 16-byte aligned.
  * It runs the same transform code as kq_quantize, so kq_quantize's codes are
@@ -197,6 +218,17 @@ int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void
 int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
                   const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, float* Y,
                   void* stream);
+
+/*
+ * kq_gemm_mxfp4_rank1 -- kq_gemm_mxfp4 plus the rank-1 term that restores
+ * the centring variant's offsets: Y = MXFP4(A) MXFP4(B)^T + mu wsum^T, with
+ * mu [M] the offsets given to kq_quantize_centered and wsum [N] = W 1 the
+ * row sums of the unfolded weights (both fp32, 4-byte aligned); the term is
+ * added in fp32 in the epilogue.  Other arguments as kq_gemm_mxfp4.
+ */
+int kq_gemm_mxfp4_rank1(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                        const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K,
+                        const float* mu, const float* wsum, float* Y, void* stream);
 
 /*
  * kq_dequant -- MXFP4 back to fp32, for checking:

@@ -273,6 +273,29 @@ def quantize_weights(W: np.ndarray, params: np.ndarray):
     return quantize_mxfp4(fold_weights(W, params))
 
 
+def row_sum(x: np.ndarray, scale: float = 1.0) -> np.ndarray:
+    """scale * sum over the row of x (fp64): the per-token mean with
+    scale = 1/d, the weight row sums W 1 with scale = 1."""
+    return scale * np.sum(np.asarray(x, dtype=np.float64), axis=1)
+
+
+def quantize_centered(x: np.ndarray, params: np.ndarray, mu: np.ndarray):
+    """[centering variant] the quantizer applied to the centred tokens:
+    MXFP4(T (x - mu 1)) for each token row with its own offset mu (the
+    per-token mean in the variant; any per-token constant restores exactly)."""
+    x = np.asarray(x, dtype=np.float64)
+    return quantize_mxfp4(transform(x - np.asarray(mu, dtype=np.float64)[:, None], params))
+
+
+def gemm_mxfp4_rank1(codes_a, scales_a, codes_b, scales_b, mu, wsum) -> np.ndarray:
+    """The layer on centred activations with the removed mean restored in
+    full precision: Y = MXFP4(A) MXFP4(B)^T + mu wsum^T, where mu [M] are the
+    per-token offsets and wsum [N] = W 1 the row sums of the unfolded weights:
+    (x - mu 1) W^T + mu (W 1)^T = x W^T."""
+    return gemm_mxfp4(codes_a, scales_a, codes_b, scales_b) + np.outer(
+        np.asarray(mu, dtype=np.float64), np.asarray(wsum, dtype=np.float64))
+
+
 def gemm_mxfp4(codes_a, scales_a, codes_b, scales_b) -> np.ndarray:
     """[ABS] the W4A4 linear layer on the quantised operands: every MXFP4
     value decoded (E2M1 code times its block's E8M0 scale), then

@@ -391,6 +391,30 @@ def pin_gemm_mxfp4_by_hand(o):
     assert t[1, 1, 16 * 1 + 3] == sc[129, 7] and t[1, 0, 16 * 2] == 0
 
 
+def pin_centering(o):
+    """Shifting every token by its own constant changes nothing after
+    centring (the shift is exact in fp64 here: dyadic values); the rank-1
+    term restores the layer exactly without quantisation: with the
+    quantised operands replaced by their exact values, (x - mu 1) W'^T-side
+    plus mu (W 1) is x W^T."""
+    rng = np.random.default_rng(51)
+    M, d, N = 6, 96, 5
+    x = np.round(rng.normal(size=(M, d)) * 64) / 64
+    p = _rand_params(d // 32, seed=52)
+    mu = o.row_sum(x, 1.0 / d)
+    assert np.allclose(mu, x.mean(axis=1), rtol=0, atol=1e-15)
+    shift = np.round(rng.normal(size=M) * 8) / 8
+    c1, s1 = o.quantize_centered(x, p, mu)
+    c2, s2 = o.quantize_centered(x + shift[:, None], p, mu + shift)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    W = rng.normal(size=(N, d))
+    wsum = o.row_sum(W)
+    xt = o.transform(x - mu[:, None], p)                   # exact transformed, centred tokens
+    Wt = o.fold_weights(W, p)
+    lhs = xt @ Wt.T + np.outer(mu, wsum)
+    assert np.allclose(lhs, x @ W.T, rtol=1e-10, atol=1e-10 * np.abs(x @ W.T).max())
+
+
 def pin_smoothquant_is_diagonal_case(o):
     """a = b = 0 makes T diagonal; SmoothQuant with 1/s = diag(T) then gives
     the same codes and scales."""

@@ -28,7 +28,8 @@ def header_functions():
 
 def test_header_declares_the_abi():
     names = header_functions()
-    for want in ("kq_quantize", "kq_quantize_sf_tiled", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
+    for want in ("kq_quantize", "kq_quantize_sf_tiled", "kq_quantize_centered", "kq_row_sum",
+                 "kq_gemm_mxfp4_rank1", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
                  "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4",
                  "kq_dequant", "kq_status_string",
                  "kq_device_status"):
@@ -110,6 +111,11 @@ def test_other_argument_checks(lib):
     assert lib.kq_quantize_weights(A16, 4, 64, None, A16c, A16d, None) == 1
     assert lib.kq_quantize_weights(None, 0, 64, None, None, None, None) == 0
     assert lib.kq_sf_tile(A16, 4, 96, A16b, None) == 1                  # K % 128
+    assert lib.kq_quantize_centered(A16, 0, 4, 64, A16b, None, A16c, A16d, None) == 1   # NULL mu
+    assert lib.kq_quantize_centered(A16, 0, 4, 64, A16b, A16 + 2, A16c, A16d, None) == 2
+    assert lib.kq_row_sum(A16, 2, 4, 64, 1.0, A16b, None) == 3
+    assert lib.kq_row_sum(A16 + 8, 0, 4, 64, 1.0, A16b, None) == 2
+    assert lib.kq_gemm_mxfp4_rank1(A16, A16b, A16c, A16d, 128, 128, 256, None, A16, A16, None) == 1
     assert lib.kq_quantize_sf_tiled(A16, 0, 4, 96, A16b, A16c, A16d, None) == 1   # d % 128
     assert lib.kq_quantize_sf_tiled(None, 0, 0, 128, None, None, None, None) == 0
     assert lib.kq_sf_tile(None, 0, 128, None, None) == 0

@@ -147,6 +147,11 @@ def m_weights_folded_with_forward(o):
     o.quantize_weights = qw
 
 
+def m_centering_after_transform(o):
+    o.quantize_centered = lambda x, params, mu: o.quantize_mxfp4(
+        o.transform(np.asarray(x, dtype=np.float64), params) - np.asarray(mu, dtype=np.float64)[:, None])
+
+
 MUTANTS = [v for k, v in sorted(globals().items()) if k.startswith("m_")]
 
 

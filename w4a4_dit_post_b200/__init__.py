@@ -19,8 +19,10 @@ import torch
 from .build import LIB_PATH
 
 __all__ = [
-    "abi", "kq_quantize", "kq_quantize_sf_tiled", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
-    "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4", "kq_dequant",
+    "abi", "kq_quantize", "kq_quantize_sf_tiled", "kq_quantize_centered", "kq_row_sum",
+    "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
+    "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4", "kq_gemm_mxfp4_rank1",
+    "kq_dequant",
     "kq_device_status",
     "kq_selftest_bounded_wait",
     "KroQuantError",
@@ -51,6 +53,11 @@ _SIGNATURES = {
     "kq_fold_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
     "kq_quantize_weights": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_sf_tile": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
+    "kq_quantize_centered": (_int, [_c_void_p, _int, _i64, _i64, _c_void_p, _c_void_p, _c_void_p,
+                                    _c_void_p, _c_void_p]),
+    "kq_row_sum": (_int, [_c_void_p, _int, _i64, _i64, ctypes.c_float, _c_void_p, _c_void_p]),
+    "kq_gemm_mxfp4_rank1": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
+                                   _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_gemm_mxfp4": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _c_void_p,
                              _c_void_p]),
     "kq_dequant": (_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
@@ -275,6 +282,55 @@ def kq_gemm_mxfp4(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
         _check("kq_gemm_mxfp4", abi().kq_gemm_mxfp4(
             a_codes.data_ptr(), a_sf_tiled.data_ptr(), b_codes.data_ptr(), b_sf_tiled.data_ptr(),
             M, N, K, Y.data_ptr(), _stream(a_codes)))
+    return Y
+
+
+def kq_row_sum(x, scale=1.0, out=None):
+    """out [M] fp32 = scale * row sums of x [M, d] (bf16 or fp32)."""
+    _need_cuda("x", x, _ACT, 2)
+    M, d = x.shape
+    out = _out(out, (M,), torch.float32, x, "out")
+    with torch.cuda.device(x.device):
+        _check("kq_row_sum", abi().kq_row_sum(x.data_ptr(), _x_dtype(x), M, d, float(scale),
+                                              out.data_ptr(), _stream(x)))
+    return out
+
+
+def kq_quantize_centered(x, params, mu, codes=None, scales=None):
+    """Centring variant: MXFP4(T (x - mu 1)) with mu [M] fp32 per-token offsets."""
+    _need_cuda("x", x, _ACT, 2)
+    _need_cuda("params", params, (torch.float32,))
+    _need_cuda("mu", mu, (torch.float32,), 1)
+    M, d = x.shape
+    if mu.shape[0] != M:
+        raise ValueError("mu must have one offset per row of x")
+    codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
+    scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
+    with torch.cuda.device(x.device):
+        _check("kq_quantize_centered", abi().kq_quantize_centered(
+            x.data_ptr(), _x_dtype(x), M, d, params.data_ptr(), mu.data_ptr(), codes.data_ptr(),
+            scales.data_ptr(), _stream(x)))
+    return codes, scales
+
+
+def kq_gemm_mxfp4_rank1(a_codes, a_sf_tiled, b_codes, b_sf_tiled, mu, wsum, Y=None):
+    """kq_gemm_mxfp4 plus mu wsum^T (mu [M], wsum [N] fp32)."""
+    for name, t in (("a_codes", a_codes), ("b_codes", b_codes)):
+        _need_cuda(name, t, (torch.uint8,), 2)
+    for name, t in (("a_sf_tiled", a_sf_tiled), ("b_sf_tiled", b_sf_tiled)):
+        _need_cuda(name, t, (torch.uint8,), 3)
+    _need_cuda("mu", mu, (torch.float32,), 1)
+    _need_cuda("wsum", wsum, (torch.float32,), 1)
+    M, half = a_codes.shape
+    N = b_codes.shape[0]
+    K = 2 * half
+    if b_codes.shape[1] != half or mu.shape[0] != M or wsum.shape[0] != N:
+        raise ValueError("operand shapes disagree")
+    Y = _out(Y, (M, N), torch.float32, a_codes, "Y")
+    with torch.cuda.device(a_codes.device):
+        _check("kq_gemm_mxfp4_rank1", abi().kq_gemm_mxfp4_rank1(
+            a_codes.data_ptr(), a_sf_tiled.data_ptr(), b_codes.data_ptr(), b_sf_tiled.data_ptr(),
+            M, N, K, mu.data_ptr(), wsum.data_ptr(), Y.data_ptr(), _stream(a_codes)))
     return Y
 
 

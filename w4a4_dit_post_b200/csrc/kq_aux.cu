@@ -127,6 +127,36 @@ fold_quant_kernel(const float* __restrict__ W, const float* __restrict__ params,
   }
 }
 
+// out[r] = scale * sum of row r (bf16 or fp32 input, fp32 accumulation):
+// one warp per row, 16-byte loads.
+__global__ void __launch_bounds__(kAuxThreads)
+row_sum_kernel(const void* __restrict__ x, int bf16, int M, int d, float scale, float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < M; r += warps) {
+    float acc = 0.0f;
+    if (bf16) {
+      const uint4* row = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)r * d);
+      for (int i = lane; i < d / 8; i += 32) {
+        const uint4 w = row[i];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          acc += __uint_as_float(ws[e] << 16) + __uint_as_float(ws[e] & 0xffff0000u);
+      }
+    } else {
+      const float4* row = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)r * d);
+      for (int i = lane; i < d / 4; i += 32) {
+        const float4 f = row[i];
+        acc += (f.x + f.y) + (f.z + f.w);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) out[r] = acc * scale;
+  }
+}
+
 // E2M1 magnitude of a 3-bit code: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
 __device__ __forceinline__ float e2m1_mag(uint32_t c) {
   // exponent field e = c >> 1, mantissa bit m = c & 1:
@@ -234,6 +264,20 @@ int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* param
   kq::fold_quant_kernel<<<kq::grid_for((int)lanes), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
       W, params, nb, n_blocks, codes, scales, devstat);
   return kq::check_launch("fold_quant_kernel launch");
+}
+
+int kq_row_sum(const void* x, int x_dtype, int64_t M, int64_t d, float scale, float* out, void* stream) {
+  if (int st = kq::check_shape(M, d, 0, "kq_row_sum")) return st;
+  if (x_dtype != KQ_DTYPE_BF16 && x_dtype != KQ_DTYPE_F32)
+    return kq::fail(KQ_ERR_DTYPE, "kq_row_sum: x_dtype = %d", x_dtype);
+  if (M == 0) return KQ_OK;
+  if (!x || !out) return kq::fail(KQ_ERR_INVALID_ARG, "kq_row_sum: NULL pointer");
+  if (!kq::aligned(x, 16) || !kq::aligned(out, 4))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_row_sum: x must be 16-byte and out 4-byte aligned");
+  const int64_t lanes = M * 32;
+  kq::row_sum_kernel<<<kq::grid_for(lanes > (1 << 30) ? (1 << 30) : (int)lanes), kq::kAuxThreads, 0,
+                       kq::as_stream(stream)>>>(x, x_dtype == KQ_DTYPE_BF16, (int)M, (int)d, scale, out);
+  return kq::check_launch("row_sum_kernel launch");
 }
 
 int kq_dequant(const uint8_t* codes, const uint8_t* scales, int64_t M, int64_t d, float* out,

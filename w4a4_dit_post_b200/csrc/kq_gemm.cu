@@ -151,6 +151,8 @@ struct GemmArgs {
   const uint8_t* sfb;        // blocked scales of B
   int m_tiles, n_tiles;
   float* Y;                  // [M][N] fp32
+  const float* mu;           // optional rank-1 term: Y += mu wsum^T (mu [M], wsum [N])
+  const float* wsum;
   int tma_store;             // 1: Y leaves through shared memory and TMA stores (N % 4 == 0)
 };
 
@@ -306,6 +308,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
       for (int c = 0; c < kTile / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+        if (args.mu != nullptr) {
+          // the centring variant's removed mean, restored in fp32
+          const float m = row < args.M ? args.mu[row] : 0.0f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int col = n0 + 32 * c + k;
+            const float ws = col < args.N ? __ldg(args.wsum + col) : 0.0f;
+            r[k] = __float_as_uint(__fmaf_rn(m, ws, __uint_as_float(r[k])));
+          }
+        }
         if (c == kTile / 32 - 1) {
           // the whole accumulator is in registers or staged: hand it back
           fence_before_sync();
@@ -399,30 +411,12 @@ constexpr int kMaxDevices = 64;
 }  // namespace
 }  // namespace kq
 
-extern "C" {
+namespace kq {
 
-int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void* stream) {
-  const char* fn = "kq_sf_tile";
-  if (R < 0 || K <= 0 || K % 128 != 0)
-    return kq::fail(KQ_ERR_INVALID_ARG, "%s: need R >= 0 and K a positive multiple of 128 (K = %lld)", fn,
-                    (long long)K);
-  if (R == 0) return KQ_OK;
-  if (!scales || !tiled) return kq::fail(KQ_ERR_INVALID_ARG, "%s: NULL pointer", fn);
-  const int64_t n_out = (R + 127) / 128 * (K / 128) * 512;
-  if (n_out >= ((int64_t)1 << 31) || R * (K / 32) >= ((int64_t)1 << 31))
-    return kq::fail(KQ_ERR_UNSUPPORTED, "%s: too large", fn);
-  int sms = 0;
-  if (int st = kq::sm_count(&sms)) return st;
-  int64_t blocks = (n_out + 255) / 256;
-  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-  kq::gemm::sf_tile_kernel<<<(unsigned)blocks, 256, 0, kq::as_stream(stream)>>>(
-      scales, (int)R, (int)(K / 32), (int)n_out, tiled);
-  return kq::check_launch("sf_tile_kernel launch");
-}
-
-int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
-                  const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, float* Y, void* stream) {
-  const char* fn = "kq_gemm_mxfp4";
+// Shared by kq_gemm_mxfp4 (mu = wsum = NULL) and kq_gemm_mxfp4_rank1.
+int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, const float* mu,
+                const float* wsum, float* Y, void* stream, const char* fn) {
   if (M < 0 || N < 0 || K <= 0 || K % 128 != 0)
     return kq::fail(KQ_ERR_INVALID_ARG, "%s: need M, N >= 0 and K a positive multiple of 128", fn);
   if (M == 0 || N == 0) return KQ_OK;
@@ -476,6 +470,8 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   args.tma_store = tma_store ? 1 : 0;
   args.m_tiles = (int)((M + 127) / 128);
   args.n_tiles = (int)((N + 127) / 128);
+  args.mu = mu;
+  args.wsum = wsum;
   unsigned int* devstat = nullptr;
   if (int st = kq::device_status_address(&devstat)) return st;
 
@@ -496,6 +492,46 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
   err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel, am, bm, ym, args, devstat);
   if (err != cudaSuccess) return kq::cuda_fail(err, "gemm_kernel launch");
   return kq::check_launch("gemm_kernel launch");
+}
+
+}  // namespace kq
+
+extern "C" {
+
+int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void* stream) {
+  const char* fn = "kq_sf_tile";
+  if (R < 0 || K <= 0 || K % 128 != 0)
+    return kq::fail(KQ_ERR_INVALID_ARG, "%s: need R >= 0 and K a positive multiple of 128 (K = %lld)", fn,
+                    (long long)K);
+  if (R == 0) return KQ_OK;
+  if (!scales || !tiled) return kq::fail(KQ_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  const int64_t n_out = (R + 127) / 128 * (K / 128) * 512;
+  if (n_out >= ((int64_t)1 << 31) || R * (K / 32) >= ((int64_t)1 << 31))
+    return kq::fail(KQ_ERR_UNSUPPORTED, "%s: too large", fn);
+  int sms = 0;
+  if (int st = kq::sm_count(&sms)) return st;
+  int64_t blocks = (n_out + 255) / 256;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  kq::gemm::sf_tile_kernel<<<(unsigned)blocks, 256, 0, kq::as_stream(stream)>>>(
+      scales, (int)R, (int)(K / 32), (int)n_out, tiled);
+  return kq::check_launch("sf_tile_kernel launch");
+}
+
+int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                  const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, float* Y, void* stream) {
+  return kq::gemm_launch(a_codes, a_sf_tiled, b_codes, b_sf_tiled, M, N, K, nullptr, nullptr, Y, stream,
+                         "kq_gemm_mxfp4");
+}
+
+int kq_gemm_mxfp4_rank1(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                        const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, const float* mu,
+                        const float* wsum, float* Y, void* stream) {
+  if (M > 0 && N > 0 && (!mu || !wsum))
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_gemm_mxfp4_rank1: NULL mu or wsum");
+  if ((mu && !kq::aligned(mu, 4)) || (wsum && !kq::aligned(wsum, 4)))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_gemm_mxfp4_rank1: mu and wsum must be 4-byte aligned");
+  return kq::gemm_launch(a_codes, a_sf_tiled, b_codes, b_sf_tiled, M, N, K, mu, wsum, Y, stream,
+                         "kq_gemm_mxfp4_rank1");
 }
 
 }  // extern "C"

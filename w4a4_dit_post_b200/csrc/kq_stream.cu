@@ -241,7 +241,7 @@ template <int kInBytes, Op kOp>
 __global__ void __launch_bounds__(kThreads, 2)
 stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ coef_src,
               const Geometry geo, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-              float* __restrict__ y_out) {
+              float* __restrict__ y_out, const float* __restrict__ mu) {
   constexpr int kStages = StageCfg<kInBytes>::kStages;
   constexpr int kRow = Table<kOp>::kRowFloats;
 
@@ -355,9 +355,24 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
     const int s = k % kStages;
     const uint32_t parity = (uint32_t)(k / kStages) & 1u;
     float2 v[32];
+    // centring variant: this row pair's offsets (read before the wait, so
+    // the load overlaps it)
+    float2 neg_mu = make_float2(0.0f, 0.0f);
+    if (kOp == Op::kKqQuant && mu != nullptr && active) {
+      const int r = rt * R + 2 * rp;
+      neg_mu = make_float2(r < geo.M ? -mu[r] : 0.0f, r + 1 < geo.M ? -mu[r + 1] : 0.0f);
+    }
     const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity);
     if (ok) {
-      if (active) load_pair<kInBytes>(smem + s * stage_bytes, C, rp, c, v);
+      if (active) {
+        load_pair<kInBytes>(smem + s * stage_bytes, C, rp, c, v);
+        if constexpr (kOp == Op::kKqQuant) {
+          if (mu != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __fadd2_rn(v[i], neg_mu);
+          }
+        }
+      }
     } else {
       *abort_flag = 1;
       atomicOr(&g_devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
@@ -481,7 +496,7 @@ constexpr int kMaxDevices = 64;
 
 template <int kInBytes, Op kOp>
 int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_t* codes,
-                  uint8_t* scales, float* y, cudaStream_t stream, bool sf_tiled) {
+                  uint8_t* scales, float* y, cudaStream_t stream, bool sf_tiled, const float* mu) {
   const int nb = (int)(d / 32);
   Geometry geo = make_geometry<kInBytes>(M, nb);
   geo.sf_tiled = sf_tiled ? 1 : 0;
@@ -529,7 +544,7 @@ int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kern, tm, coef, geo, codes, scales, y);
+  err = cudaLaunchKernelEx(&cfg, kern, tm, coef, geo, codes, scales, y, mu);
   if (err != cudaSuccess) return cuda_fail(err, "stream_kernel launch");
   return check_launch("stream_kernel launch");
 }
@@ -537,7 +552,7 @@ int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_
 template <Op kOp>
 int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef,
              uint8_t* codes, uint8_t* scales, float* y, void* stream, const char* fn,
-             bool sf_tiled = false) {
+             bool sf_tiled = false, const float* mu = nullptr, bool need_mu = false) {
   if (int st = check_shape(M, d, KQ_MAX_D, fn)) return st;
   if (sf_tiled && d % 128 != 0)
     return fail(KQ_ERR_INVALID_ARG, "%s: d must be a multiple of 128 (d = %lld)", fn, (long long)d);
@@ -550,13 +565,15 @@ int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef
   } else if (!codes || !scales) {
     return fail(KQ_ERR_INVALID_ARG, "%s: NULL output pointer", fn);
   }
+  if (need_mu && !mu) return fail(KQ_ERR_INVALID_ARG, "%s: NULL mu", fn);
+  if (mu && !aligned(mu, 4)) return fail(KQ_ERR_ALIGNMENT, "%s: mu must be 4-byte aligned", fn);
   if (!aligned(x, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: x must be 16-byte aligned", fn);
   if (!aligned(coef, 4)) return fail(KQ_ERR_ALIGNMENT, "%s: parameters must be 4-byte aligned", fn);
   if (codes && !aligned(codes, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: codes must be 16-byte aligned", fn);
   if (y && !aligned(y, 16)) return fail(KQ_ERR_ALIGNMENT, "%s: y must be 16-byte aligned", fn);
   const cudaStream_t s = as_stream(stream);
-  if (x_dtype == KQ_DTYPE_BF16) return launch_stream<2, kOp>(x, M, d, coef, codes, scales, y, s, sf_tiled);
-  return launch_stream<4, kOp>(x, M, d, coef, codes, scales, y, s, sf_tiled);
+  if (x_dtype == KQ_DTYPE_BF16) return launch_stream<2, kOp>(x, M, d, coef, codes, scales, y, s, sf_tiled, mu);
+  return launch_stream<4, kOp>(x, M, d, coef, codes, scales, y, s, sf_tiled, mu);
 }
 
 }  // namespace
@@ -590,6 +607,12 @@ int kq_quantize(const void* x, int x_dtype, int64_t M, int64_t d, const float* p
                 uint8_t* codes, uint8_t* scales, void* stream) {
   return kq::dispatch<kq::Op::kKqQuant>(x, x_dtype, M, d, params, codes, scales, nullptr, stream,
                                         "kq_quantize");
+}
+
+int kq_quantize_centered(const void* x, int x_dtype, int64_t M, int64_t d, const float* params,
+                         const float* mu, uint8_t* codes, uint8_t* scales, void* stream) {
+  return kq::dispatch<kq::Op::kKqQuant>(x, x_dtype, M, d, params, codes, scales, nullptr, stream,
+                                        "kq_quantize_centered", false, mu, true);
 }
 
 int kq_quantize_sf_tiled(const void* x, int x_dtype, int64_t M, int64_t d, const float* params,
