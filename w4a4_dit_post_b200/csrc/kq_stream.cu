@@ -237,7 +237,51 @@ __device__ __forceinline__ uint4 lane_codes(const float2 (&r)[32]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <int kInBytes, Op kOp>
+// Transform of one row pair of one block column and its output: the
+// transformed values (kq_transform), or the E2M1 codes and E8M0 scale bytes.
+// Rows r0 and r0 + 1 (the second only when `second`), block column jc; g0 =
+// r0 * nb + jc is the flat block index, and cdst, sdst, ydst point at block
+// g0 of codes, scales and y.
+template <Op kOp>
+__device__ __forceinline__ void quantize_pair(float2 (&v)[32], const float* crow, const Geometry& geo,
+                                              int r0, bool second, int jc, uint8_t* cdst,
+                                              uint8_t* sdst, float* ydst, uint8_t* __restrict__ scales) {
+  const int nb = geo.nb;
+  if constexpr (kOp == Op::kSqQuant) {
+    sq_transform_pair(v, crow);
+  } else {
+    kq_transform_pair(v, crow);
+  }
+  if constexpr (kOp == Op::kKqTransform) {
+    float4* d0 = reinterpret_cast<float4*>(ydst);
+    float4* d1 = reinterpret_cast<float4*>(ydst + (size_t)nb * 32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      d0[q] = make_float4(v[4 * q].x, v[4 * q + 1].x, v[4 * q + 2].x, v[4 * q + 3].x);
+      if (second)
+        d1[q] = make_float4(v[4 * q].y, v[4 * q + 1].y, v[4 * q + 2].y, v[4 * q + 3].y);
+    }
+  } else {
+    const uint32_t e0 = e8m0_byte(lane_absmax<0>(v));
+    const uint32_t e1 = e8m0_byte(lane_absmax<1>(v));
+    const float2 sc = make_float2(inv_scale_from_byte(e0), inv_scale_from_byte(e1));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], sc);
+    *reinterpret_cast<uint4*>(cdst) = lane_codes<0>(v);
+    if (geo.sf_tiled) {
+      scales[sf_tiled_offset(r0, jc, nb)] = (uint8_t)e0;
+      if (second) scales[sf_tiled_offset(r0 + 1, jc, nb)] = (uint8_t)e1;
+    } else {
+      sdst[0] = (uint8_t)e0;
+      if (second) sdst[nb] = (uint8_t)e1;
+    }
+    if (second) *reinterpret_cast<uint4*>(cdst + (size_t)nb * 16) = lane_codes<1>(v);
+  }
+}
+
+// kC: the column-group width when it is fixed at compile time (32, every
+// d that is a multiple of 1024), else 0 and the width comes from geo.
+template <int kInBytes, Op kOp, int kC>
 __global__ void __launch_bounds__(kThreads, 2)
 stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ coef_src,
               const Geometry geo, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -248,13 +292,16 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const int stage_bytes = geo.stage_bytes;
+  // with a fixed group width the tile geometry is a compile-time constant
+  const int stage_bytes = kC ? ((2 * (kThreads / (kC ? kC : 1)) * kC * InLayout<kInBytes>::kBlockBytes + 1023) & ~1023)
+                             : geo.stage_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes);
   int* abort_flag = reinterpret_cast<int*>(smem + kStages * stage_bytes + 8 * kStages);
   float* table = reinterpret_cast<float*>(smem + kStages * stage_bytes + 128);
 
   const int tid = threadIdx.x;
-  const int C = geo.C, R = geo.R;
+  __builtin_assume(tid < kThreads);
+  const int C = kC ? kC : geo.C, R = kC ? 2 * (kThreads / (kC ? kC : 1)) : geo.R;
   const int col_group = blockIdx.x % geo.NC;
   const int row_step = gridDim.x / geo.NC;      // CTAs sharing this column group
   const int rt_first = blockIdx.x / geo.NC;
@@ -350,89 +397,75 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   const float* crow = table + c * kRow;
   const int nb = geo.nb;
 
-  int k = 0;
-  for (int rt = rt_first; rt < geo.n_row_tiles; rt += row_step, ++k) {
-    const int s = k % kStages;
-    const uint32_t parity = (uint32_t)(k / kStages) & 1u;
-    float2 v[32];
-    // centring variant: this row pair's offsets (read before the wait, so
-    // the load overlaps it)
-    float2 neg_mu = make_float2(0.0f, 0.0f);
-    if (kOp == Op::kKqQuant && mu != nullptr && active) {
-      const int r = rt * R + 2 * rp;
-      neg_mu = make_float2(r < geo.M ? -mu[r] : 0.0f, r + 1 < geo.M ? -mu[r + 1] : 0.0f);
-    }
-    const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity);
-    if (ok) {
-      if (active) {
-        load_pair<kInBytes>(smem + s * stage_bytes, C, rp, c, v);
-        if constexpr (kOp == Op::kKqQuant) {
-          if (mu != nullptr) {
+  // Tiles walk the stages in order; the barrier phase flips once per round of
+  // kStages tiles (a counter and a flag instead of a division per tile).
+  // Unrolling this loop over the stages made ptxas spill.
+  int rt = rt_first;
+  uint32_t parity = 0;
+  // this thread's first row, and its output blocks, advanced by a constant per tile
+  int r0 = rt_first * R + 2 * rp;
+  const int r_step = row_step * R;
+  const size_t g_first = (size_t)r0 * nb + j0 + c, g_step = (size_t)r_step * nb;
+  constexpr bool kCodes = kOp != Op::kKqTransform;   // the other output is NULL
+  uint8_t* cdst = kCodes ? codes + g_first * 16 : nullptr;
+  uint8_t* sdst = kCodes ? scales + g_first : nullptr;
+  float* ydst = kCodes ? nullptr : y_out + g_first * 32;
+  for (;;) {
+#pragma unroll 1
+    for (int s = 0; s < kStages; ++s, rt += row_step, r0 += r_step) {
+      if (rt >= geo.n_row_tiles) return;
+      float2 v[32];
+      // centring variant: this row pair's offsets (read before the wait, so
+      // the load overlaps it)
+      float2 neg_mu = make_float2(0.0f, 0.0f);
+      if (kOp == Op::kKqQuant && mu != nullptr && active)
+        neg_mu = make_float2(r0 < geo.M ? -mu[r0] : 0.0f, r0 + 1 < geo.M ? -mu[r0 + 1] : 0.0f);
+      const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity);
+      if (ok) {
+        if (active) {
+          load_pair<kInBytes>(smem + s * stage_bytes, C, rp, c, v);
+          if constexpr (kOp == Op::kKqQuant) {
+            if (mu != nullptr) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __fadd2_rn(v[i], neg_mu);
+              for (int i = 0; i < 32; ++i) v[i] = __fadd2_rn(v[i], neg_mu);
+            }
           }
         }
+      } else {
+        *abort_flag = 1;
+        atomicOr(&g_devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
       }
-    } else {
-      *abort_flag = 1;
-      atomicOr(&g_devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
-    }
-    __syncthreads();
-    if (*abort_flag) {
-      // let the loads still in flight land before shared memory goes away
+      __syncthreads();
+      if (*abort_flag) {
+        // let the loads still in flight land before shared memory goes away:
+        // this tile's and the next kStages - 1, in the following stages
+        if (tid == 0) {
+          for (int i = 0; i < kStages; ++i) {
+            if (rt + i * row_step >= geo.n_row_tiles) break;
+            const int si = (s + i) % kStages;
+            const uint32_t pi = parity ^ (uint32_t)((s + i) / kStages);
+            (void)mbar_wait_bounded(smem_addr(&bars[si]), pi & 1u);
+          }
+        }
+        return;
+      }
       if (tid == 0) {
-        for (int kk = k; kk < k + kStages; ++kk) {
-          if (rt_first + kk * row_step >= geo.n_row_tiles) break;
-          (void)mbar_wait_bounded(smem_addr(&bars[kk % kStages]), (uint32_t)(kk / kStages) & 1u);
+        const int nrt = rt + kStages * row_step;
+        if (nrt < geo.n_row_tiles) {
+          mbar_arrive_expect_tx(smem_addr(&bars[s]), tile_tx);
+          tma_load_3d(smem_addr(smem + s * stage_bytes), &tmap, 0, j0, nrt * R, smem_addr(&bars[s]));
         }
       }
-      return;
-    }
-    if (tid == 0) {
-      const int nrt = rt + kStages * row_step;
-      if (nrt < geo.n_row_tiles) {
-        mbar_arrive_expect_tx(smem_addr(&bars[s]), tile_tx);
-        tma_load_3d(smem_addr(smem + s * stage_bytes), &tmap, 0, j0, nrt * R, smem_addr(&bars[s]));
-      }
-    }
-    if (!active) continue;
-
-    const int r0 = rt * R + 2 * rp;             // rows r0 and r0 + 1
-    if (r0 >= geo.M) continue;
-    const bool second = r0 + 1 < geo.M;
-    const size_t g0 = (size_t)r0 * nb + j0 + c; // flat block index of (r0, column)
-
-    if constexpr (kOp == Op::kSqQuant) {
-      sq_transform_pair(v, crow);
-    } else {
-      kq_transform_pair(v, crow);
-    }
-
-    if constexpr (kOp == Op::kKqTransform) {
-      float4* d0 = reinterpret_cast<float4*>(y_out + g0 * 32);
-      float4* d1 = reinterpret_cast<float4*>(y_out + (g0 + nb) * 32);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        d0[q] = make_float4(v[4 * q].x, v[4 * q + 1].x, v[4 * q + 2].x, v[4 * q + 3].x);
-        if (second)
-          d1[q] = make_float4(v[4 * q].y, v[4 * q + 1].y, v[4 * q + 2].y, v[4 * q + 3].y);
-      }
-    } else {
-      const uint32_t e0 = e8m0_byte(lane_absmax<0>(v));
-      const uint32_t e1 = e8m0_byte(lane_absmax<1>(v));
-      const float2 sc = make_float2(inv_scale_from_byte(e0), inv_scale_from_byte(e1));
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], sc);
-      *reinterpret_cast<uint4*>(codes + g0 * 16) = lane_codes<0>(v);
-      if (geo.sf_tiled) {
-        scales[sf_tiled_offset(r0, j0 + c, nb)] = (uint8_t)e0;
-        if (second) scales[sf_tiled_offset(r0 + 1, j0 + c, nb)] = (uint8_t)e1;
+      if (active && r0 < geo.M)                   // rows r0 and r0 + 1
+        quantize_pair<kOp>(v, crow, geo, r0, r0 + 1 < geo.M, j0 + c, cdst, sdst, ydst, scales);
+      if constexpr (kCodes) {
+        cdst += g_step * 16;
+        sdst += g_step;
       } else {
-        scales[g0] = (uint8_t)e0;
-        if (second) scales[g0 + nb] = (uint8_t)e1;
+        ydst += g_step * 32;
       }
-      if (second) *reinterpret_cast<uint4*>(codes + (g0 + nb) * 16) = lane_codes<1>(v);
     }
+    parity ^= 1u;
   }
 }
 
@@ -500,21 +533,26 @@ int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_
   const int nb = (int)(d / 32);
   Geometry geo = make_geometry<kInBytes>(M, nb);
   geo.sf_tiled = sf_tiled ? 1 : 0;
-  auto kern = stream_kernel<kInBytes, kOp>;
+  auto kern = geo.C == 32 ? stream_kernel<kInBytes, kOp, 32> : stream_kernel<kInBytes, kOp, 0>;
   const size_t smem = smem_bytes<kInBytes, kOp>(geo);
 
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
-  // per device and instantiation: allow the largest dynamic shared memory once
+  // per device and instantiation (both group-width variants): allow the
+  // largest dynamic shared memory once
   static std::once_flag attr_once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
   std::call_once(attr_once[dev], [&] {
     int optin = 0;
     attr_err[dev] = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (attr_err[dev] == cudaSuccess)
-      attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+      attr_err[dev] = cudaFuncSetAttribute(stream_kernel<kInBytes, kOp, 32>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (attr_err[dev] == cudaSuccess)
+      attr_err[dev] = cudaFuncSetAttribute(stream_kernel<kInBytes, kOp, 0>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
 
