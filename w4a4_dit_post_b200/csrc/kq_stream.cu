@@ -51,7 +51,8 @@ __device__ unsigned int g_devstat = 0;
 constexpr int kThreads = 256;
 constexpr int kMaxC = 32;
 
-enum class Op : int { kKqQuant = 0, kKqTransform = 1, kSqQuant = 2 };
+// kKqCentered: kq_quantize_centered (x - mu formed before the transform).
+enum class Op : int { kKqQuant = 0, kKqTransform = 1, kSqQuant = 2, kKqCentered = 3 };
 
 // Tile geometry, computed on the host and passed by value.
 struct Geometry {
@@ -296,7 +297,6 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   const int stage_bytes = kC ? ((2 * (kThreads / (kC ? kC : 1)) * kC * InLayout<kInBytes>::kBlockBytes + 1023) & ~1023)
                              : geo.stage_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes);
-  int* abort_flag = reinterpret_cast<int*>(smem + kStages * stage_bytes + 8 * kStages);
   float* table = reinterpret_cast<float*>(smem + kStages * stage_bytes + 128);
 
   const int tid = threadIdx.x;
@@ -323,7 +323,6 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
     tma_prefetch_desc(&tmap);
 #pragma unroll
     for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
-    *abort_flag = 0;
     mbar_init_fence();
 #pragma unroll
     for (int s = 0; s < kStages; ++s) {
@@ -418,25 +417,22 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
       // centring variant: this row pair's offsets (read before the wait, so
       // the load overlaps it)
       float2 neg_mu = make_float2(0.0f, 0.0f);
-      if (kOp == Op::kKqQuant && mu != nullptr && active)
+      if (kOp == Op::kKqCentered && active)
         neg_mu = make_float2(r0 < geo.M ? -mu[r0] : 0.0f, r0 + 1 < geo.M ? -mu[r0 + 1] : 0.0f);
       const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity);
       if (ok) {
         if (active) {
           load_pair<kInBytes>(smem + s * stage_bytes, C, rp, c, v);
-          if constexpr (kOp == Op::kKqQuant) {
-            if (mu != nullptr) {
+          if constexpr (kOp == Op::kKqCentered) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __fadd2_rn(v[i], neg_mu);
-            }
+            for (int i = 0; i < 32; ++i) v[i] = __fadd2_rn(v[i], neg_mu);
           }
         }
       } else {
-        *abort_flag = 1;
         atomicOr(&g_devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
       }
-      __syncthreads();
-      if (*abort_flag) {
+      // one barrier per tile, which also tells every thread whether any wait ran out
+      if (__syncthreads_or(!ok)) {
         // let the loads still in flight land before shared memory goes away:
         // this tile's and the next kStages - 1, in the following stages
         if (tid == 0) {
@@ -649,8 +645,8 @@ int kq_quantize(const void* x, int x_dtype, int64_t M, int64_t d, const float* p
 
 int kq_quantize_centered(const void* x, int x_dtype, int64_t M, int64_t d, const float* params,
                          const float* mu, uint8_t* codes, uint8_t* scales, void* stream) {
-  return kq::dispatch<kq::Op::kKqQuant>(x, x_dtype, M, d, params, codes, scales, nullptr, stream,
-                                        "kq_quantize_centered", false, mu, true);
+  return kq::dispatch<kq::Op::kKqCentered>(x, x_dtype, M, d, params, codes, scales, nullptr, stream,
+                                           "kq_quantize_centered", false, mu, true);
 }
 
 int kq_quantize_sf_tiled(const void* x, int x_dtype, int64_t M, int64_t d, const float* params,
