@@ -164,7 +164,10 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // t / m_tiles), so CTAs running together share B tiles in L2).  The stage
 // ring runs on across tiles, and the accumulator is handed back to the MMA
 // lane as soon as the epilogue has read it, so the next tile's loads and MMAs
-// overlap this tile's stores; two CTAs share an SM.
+// overlap this tile's stores; two CTAs share an SM.  kRank1: the epilogue adds
+// mu[m] * wsum[n] (kq_gemm_mxfp4_rank1); a compile-time switch, so that the
+// plain GEMM's epilogue keeps its registers.
+template <bool kRank1>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
             const __grid_constant__ CUtensorMap ymap, const GemmArgs args, unsigned int* devstat) {
@@ -308,7 +311,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
       for (int c = 0; c < kTile / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
-        if (args.mu != nullptr) {
+        if constexpr (kRank1) {
           // the centring variant's removed mean, restored in fp32
           const float m = row < args.M ? args.mu[row] : 0.0f;
 #pragma unroll
@@ -437,8 +440,11 @@ int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t
   static std::once_flag attr_once[kq::kMaxDevices];
   static cudaError_t attr_err[kq::kMaxDevices];
   std::call_once(attr_once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr_err[dev] == cudaSuccess)
+      attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   });
   if (attr_err[dev] != cudaSuccess) return kq::cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
 
@@ -489,7 +495,8 @@ int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel, am, bm, ym, args, devstat);
+  err = mu != nullptr ? cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel<true>, am, bm, ym, args, devstat)
+                      : cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel<false>, am, bm, ym, args, devstat);
   if (err != cudaSuccess) return kq::cuda_fail(err, "gemm_kernel launch");
   return kq::check_launch("gemm_kernel launch");
 }
