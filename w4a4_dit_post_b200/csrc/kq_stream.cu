@@ -16,7 +16,10 @@
 // are built once, in a small shared table.  Thread t owns block column
 // t % C and the row pair (2 (t / C), 2 (t / C) + 1) of every tile: the two
 // rows share their coefficients, so every butterfly operation is one packed
-// f32x2 instruction on (row 0, row 1) with a broadcast coefficient.
+// f32x2 instruction on (row 0, row 1) with a broadcast coefficient.  The
+// kernel is also compiled with C fixed at 32 (every d that is a multiple of
+// 1024), so that tile height, stage size and the thread's block offsets are
+// constants; per tile a thread then only advances counters and pointers.
 //
 // Transform.  Each LU factor A = L U (L = [[1,0],[a,1]], U = [[u,b],[0,1/u]])
 // is split as A = S L'' U' with S = diag(u, 1/u), U' = [[1, b/u], [0, 1]] and
@@ -126,6 +129,14 @@ inline Geometry make_geometry(int64_t M, int nb) {
   g.stage_bytes = (raw + 1023) & ~1023;
   return g;
 }
+
+// Stage size of a tile when the column-group width kC is fixed at compile time
+// (the same formula as make_geometry's: R = 2 * (kThreads / C) rows).
+template <int kInBytes, int kC>
+struct FixedStageBytes {
+  static constexpr int value =
+      (2 * (kThreads / kC) * kC * InLayout<kInBytes>::kBlockBytes + 1023) & ~1023;
+};
 
 template <int kInBytes, Op kOp>
 inline size_t smem_bytes(const Geometry& g) {
@@ -294,8 +305,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   // with a fixed group width the tile geometry is a compile-time constant
-  const int stage_bytes = kC ? ((2 * (kThreads / (kC ? kC : 1)) * kC * InLayout<kInBytes>::kBlockBytes + 1023) & ~1023)
-                             : geo.stage_bytes;
+  const int stage_bytes = kC ? FixedStageBytes<kInBytes, (kC ? kC : 32)>::value : geo.stage_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes);
   float* table = reinterpret_cast<float*>(smem + kStages * stage_bytes + 128);
 
@@ -531,6 +541,8 @@ int launch_stream(const void* x, int64_t M, int64_t d, const float* coef, uint8_
   geo.sf_tiled = sf_tiled ? 1 : 0;
   auto kern = geo.C == 32 ? stream_kernel<kInBytes, kOp, 32> : stream_kernel<kInBytes, kOp, 0>;
   const size_t smem = smem_bytes<kInBytes, kOp>(geo);
+  if (geo.C == 32 && geo.stage_bytes != FixedStageBytes<kInBytes, 32>::value)
+    return fail(KQ_ERR_UNSUPPORTED, "internal: tile geometry of the fixed-width kernel disagrees with the host");
 
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
