@@ -8,8 +8,9 @@ oracle and checks that some pin fails for every one of them.
 
 Nothing here calls the oracle to produce its own expected values: the
 expected side is a closed form, a library routine (numpy.linalg, scipy,
-ml_dtypes, torch dtypes), a brute-force search written here, or a value
-worked out by hand in a comment.
+ml_dtypes, torch dtypes), a brute-force search written here, a value
+worked out by hand in a comment, or a hand-worked block in
+tests/golden/kq_hand_blocks.txt (each derived there from the definitions).
 """
 from __future__ import annotations
 
@@ -21,6 +22,7 @@ import scipy.linalg
 import torch
 
 import synthetic
+from golden_cases import hand_blocks
 
 RNG_SEED = 1234
 
@@ -447,5 +449,18 @@ def pin_undecided_flags(o):
     elem2, blk2 = o.undecided(y2, tol)
     assert blk2[0, 0] and elem2.all()
 
+
+
+def pin_golden_hand_blocks(o):
+    """The hand-worked blocks of tests/golden/kq_hand_blocks.txt: ties and
+    saturation, the Kronecker factor order (a diagonal factor on the most and on
+    the least significant index bit), five rotations on a unit vector, a power-
+    of-two amax, an all-zero block and a tiny amax.  Inputs as the kernels see
+    them (rounded to fp32)."""
+    for hb in hand_blocks():
+        x = hb.x.astype(np.float32).astype(np.float64)
+        codes, scales = o.kq_quantize(x, hb.params)
+        assert int(scales[0, 0]) == hb.scale, (hb.name, int(scales[0, 0]), hb.scale)
+        assert np.array_equal(codes, hb.codes), (hb.name, codes, hb.codes)
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -10,6 +10,7 @@ import torch
 
 import oracle.kq_oracle as o
 import synthetic
+from golden_cases import hand_blocks
 from gpu_util import device_activations, f64, guards_intact, padded_u8, sample_rows, to_device
 from parity import compare_codes, compare_transform, reference
 
@@ -121,6 +122,41 @@ def test_quantize_sweep(kq, w):
           f"kq {w.key}")
     del xd, codes, scales
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# hand-worked blocks (tests/golden/kq_hand_blocks.txt), bit for bit: every
+# decision there is an exact tie or far from a rounding or scale boundary
+# ---------------------------------------------------------------------------
+def _golden_input(hb, dtype):
+    x = torch.from_numpy(hb.x.astype(np.float32)).cuda()
+    return x.to(torch.bfloat16) if dtype == "bf16" else x
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_golden_hand_blocks(kq, dtype):
+    for hb in hand_blocks():
+        codes, scales = kq.kq_quantize(_golden_input(hb, dtype), torch.from_numpy(hb.params).cuda())
+        assert int(scales.cpu()[0, 0]) == hb.scale, hb.name
+        assert np.array_equal(codes.cpu().numpy(), hb.codes), hb.name
+
+
+def test_golden_hand_blocks_tensor_core(kq):
+    for hb in hand_blocks():
+        codes, scales = kq.kq_quantize_tc(_golden_input(hb, "bf16"), torch.from_numpy(hb.params).cuda())
+        assert int(scales.cpu()[0, 0]) == hb.scale, hb.name
+        assert np.array_equal(codes.cpu().numpy(), hb.codes), hb.name
+
+
+def test_golden_hand_blocks_smoothquant_identity(kq):
+    """With unit scales SmoothQuant is plain MXFP4: the identity-transform blocks."""
+    ones = torch.ones(32, device="cuda")
+    for hb in hand_blocks():
+        if not np.array_equal(hb.params, np.tile(np.array([0, 0, 1], np.float32), 5).reshape(1, 15)):
+            continue
+        codes, scales = kq.sq_quantize(_golden_input(hb, "f32"), ones)
+        assert int(scales.cpu()[0, 0]) == hb.scale, hb.name
+        assert np.array_equal(codes.cpu().numpy(), hb.codes), hb.name
 
 
 # ---------------------------------------------------------------------------
