@@ -307,13 +307,15 @@ def fp4_peak():
 
 
 def time_gemm(kq, device, stream, K_launches: int, W: int, shapes=None) -> dict:
-    """kq_gemm_mxfp4 on the FLUX.1-schnell layer shapes (4608 tokens): mean
-    device time of K back-to-back launches on seeded codes and scales (the
-    cost does not depend on the values)."""
+    """kq_gemm_mxfp4 (fp32 Y) and kq_gemm_mxfp4_bf16 (bf16 Y) on the
+    FLUX.1-schnell layer shapes (4608 tokens): mean device time of K
+    back-to-back launches on seeded codes and scales (the cost does not depend
+    on the values)."""
     import torch
     lib = kq.abi()
     peak, src = fp4_peak()
-    out = {"kernel": "kq_gemm_mxfp4 (tcgen05 kind::mxf4 block32, fp32 out)", "peak_tflops": round(peak, 1),
+    out = {"kernel": "kq_gemm_mxfp4 (tcgen05 kind::mxf4 block32; fp32 out, and bf16 out: kq_gemm_mxfp4_bf16)",
+           "peak_tflops": round(peak, 1),
            "peak_source": src, "shapes": {}}
     g = torch.Generator(device=device)
     g.manual_seed(7)
@@ -323,40 +325,43 @@ def time_gemm(kq, device, stream, K_launches: int, W: int, shapes=None) -> dict:
         ta = kq.kq_sf_tile(torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device=device, generator=g))
         tb = kq.kq_sf_tile(torch.randint(120, 134, (N, K // 32), dtype=torch.uint8, device=device, generator=g))
         Y = torch.empty((M, N), dtype=torch.float32, device=device)
-
-        def go():
-            st = lib.kq_gemm_mxfp4(ca.data_ptr(), ta.data_ptr(), cb.data_ptr(), tb.data_ptr(), M, N, K,
-                                   Y.data_ptr(), stream.cuda_stream)
-            if st != 0:
-                raise RuntimeError(lib.kq_last_error().decode())
-        for _ in range(W):
-            go()
-        torch.cuda.synchronize(device)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(K_launches):
-            go()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        us = e0.elapsed_time(e1) / K_launches * 1e3
-        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
-        out["shapes"][f"{M}x{N}x{K}"] = {"us": round(us, 2), "tflops": round(tf, 1),
-                                         "frac_of_peak": round(tf / peak, 4)}
-        del ca, cb, ta, tb, Y
+        Y16 = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        row = {}
+        for tag, fn, y in (("", lib.kq_gemm_mxfp4, Y), ("_bf16", lib.kq_gemm_mxfp4_bf16, Y16)):
+            def go():
+                st = fn(ca.data_ptr(), ta.data_ptr(), cb.data_ptr(), tb.data_ptr(), M, N, K,
+                        y.data_ptr(), stream.cuda_stream)
+                if st != 0:
+                    raise RuntimeError(lib.kq_last_error().decode())
+            for _ in range(W):
+                go()
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(K_launches):
+                go()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            us = e0.elapsed_time(e1) / K_launches * 1e3
+            tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            row.update({f"us{tag}": round(us, 2), f"tflops{tag}": round(tf, 1),
+                        f"frac_of_peak{tag}": round(tf / peak, 4)})
+        out["shapes"][f"{M}x{N}x{K}"] = row
+        del ca, cb, ta, tb, Y, Y16
     return out
 
 
 def time_layer(kq, device, stream, K_launches: int, W: int) -> dict:
     """One W4A4 linear layer per FLUX.1-schnell layer shape, per step:
     kq_quantize_sf_tiled on the bf16 activations (codes, and scales in the
-    GEMM's block layout) and kq_gemm_mxfp4 against weights quantised offline
-    (kq_quantize_weights),
-    against the same layer as a bf16 GEMM (torch.matmul, cuBLAS) on the
-    unquantised operands.  Mean device time of K back-to-back steps."""
+    GEMM's block layout) and kq_gemm_mxfp4_bf16 (bf16 Y, like the baseline)
+    against weights quantised offline (kq_quantize_weights), against the same
+    layer as a bf16 GEMM (torch.matmul, cuBLAS) on the unquantised operands.
+    Mean device time of K back-to-back steps."""
     import torch
     lib = kq.abi()
-    out = {"step": "kq_quantize_sf_tiled + kq_gemm_mxfp4 (weights quantised offline)",
+    out = {"step": "kq_quantize_sf_tiled + kq_gemm_mxfp4_bf16 (weights quantised offline, bf16 Y)",
            "baseline": "torch.matmul bf16 (cuBLAS), same X and W", "shapes": {}}
     for M, N, K in GEMM_SHAPES:
         wd = synthetic.Workload("layer", M, K, "bf16", "normal", 0.01, None, 100.0, 4.0, 3)
@@ -368,15 +373,15 @@ def time_layer(kq, device, stream, K_launches: int, W: int) -> dict:
         tw = kq.kq_sf_tile(sw)
         codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
         tiled = torch.empty(((M + 127) // 128, K // 128, 512), dtype=torch.uint8, device=device)
-        Y = torch.empty((M, N), dtype=torch.float32, device=device)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
         Wb = Wt.to(torch.bfloat16)
         s = stream.cuda_stream
 
         def step():
             st = lib.kq_quantize_sf_tiled(x.data_ptr(), kq.KQ_DTYPE_BF16, M, K, p.data_ptr(),
                                           codes.data_ptr(), tiled.data_ptr(), s)
-            st = st or lib.kq_gemm_mxfp4(codes.data_ptr(), tiled.data_ptr(), cw.data_ptr(), tw.data_ptr(),
-                                         M, N, K, Y.data_ptr(), s)
+            st = st or lib.kq_gemm_mxfp4_bf16(codes.data_ptr(), tiled.data_ptr(), cw.data_ptr(), tw.data_ptr(),
+                                              M, N, K, Y.data_ptr(), s)
             if st != 0:
                 raise RuntimeError(lib.kq_last_error().decode())
 
@@ -508,11 +513,11 @@ def run_kroquant(args) -> int:
 
     K, W = args.steps, args.warmup
     if args.profile == "gemm":
-        # only kq_gemm_mxfp4 launches on the first FLUX layer shape (for ncu captures)
+        # only GEMM launches (fp32 Y, then bf16 Y) on the first FLUX layer shape (for ncu captures)
         M, N, Kd = GEMM_SHAPES[0]
         r = time_gemm(kq, device, stream, K, W, shapes=[GEMM_SHAPES[0]])
         if rank == 0:
-            print(json.dumps({"profile": f"kq_gemm_mxfp4 {M}x{N}x{Kd}", "launches": W + K,
+            print(json.dumps({"profile": f"kq_gemm_mxfp4 and kq_gemm_mxfp4_bf16 {M}x{N}x{Kd}", "launches": 2 * (W + K),
                               **r["shapes"][f"{M}x{N}x{Kd}"],
                               "device_status": kq.kq_device_status(device)}), flush=True)
         return 0

@@ -220,6 +220,16 @@ int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8
                   void* stream);
 
 /*
+ * kq_gemm_mxfp4_bf16 -- kq_gemm_mxfp4 with Y written as bf16 (the dtype the
+ * next op of a DiT layer takes): each fp32 sum rounded to bf16, nearest even.
+ *   Y [M][N] bf16 row-major, 16-byte aligned; other arguments and limits as
+ *   kq_gemm_mxfp4.
+ */
+int kq_gemm_mxfp4_bf16(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                       const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, void* Y,
+                       void* stream);
+
+/*
  * kq_gemm_mxfp4_rank1 -- kq_gemm_mxfp4 plus the rank-1 term that restores
  * the centring variant's offsets: Y = MXFP4(A) MXFP4(B)^T + mu wsum^T, with
  * mu [M] the offsets given to kq_quantize_centered and wsum [N] = W 1 the

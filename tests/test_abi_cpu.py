@@ -30,7 +30,7 @@ def test_header_declares_the_abi():
     names = header_functions()
     for want in ("kq_quantize", "kq_quantize_sf_tiled", "kq_quantize_centered", "kq_row_sum",
                  "kq_gemm_mxfp4_rank1", "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
-                 "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4",
+                 "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4", "kq_gemm_mxfp4_bf16",
                  "kq_dequant", "kq_status_string",
                  "kq_device_status"):
         assert want in names

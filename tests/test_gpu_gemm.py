@@ -1,4 +1,5 @@
-"""The W4A4 GEMM on the quantised operands (kq_sf_tile + kq_gemm_mxfp4)
+"""The W4A4 GEMM on the quantised operands (kq_sf_tile + kq_gemm_mxfp4, and
+kq_gemm_mxfp4_bf16)
 against the oracle.  Operand codes and scales are seeded or come from the
 oracle's own quantizers; the GPU computes Y from them.  Needs a B200.
 """
@@ -90,6 +91,52 @@ def test_gemm_on_quantized_layer(kq):
     ref = o.gemm_mxfp4(ca, sa, cb, sb)
     tol = (w.d / 64 + 64) * 2.0 ** -23 * o.gemm_error_scale(ca, sa, cb, sb)
     assert np.all(np.abs(Y - ref) <= tol)
+
+
+# ---------------------------------------------------------------------------
+# bf16 output (kq_gemm_mxfp4_bf16): the same fp32 sums, rounded to nearest even
+# ---------------------------------------------------------------------------
+def _gemm_bf16(kq, ca, sa, cb, sb):
+    ta = kq.kq_sf_tile(_cuda(sa))
+    tb = kq.kq_sf_tile(_cuda(sb))
+    Y = kq.kq_gemm_mxfp4_bf16(_cuda(ca), ta, _cuda(cb), tb)
+    torch.cuda.synchronize()
+    return Y.cpu()
+
+
+def _bf16_bits(t):
+    return t.contiguous().view(torch.int16).numpy()
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (200, 72, 384), (256, 384, 1024), (1, 1, 128), (300, 1029, 256)])
+def test_gemm_bf16_unit_scales_is_exact(kq, M, N, K):
+    """Unit scales: the fp32 sum is the oracle's exact value, so Y is that value
+    rounded to bf16 (torch's round-to-nearest-even conversion), bit for bit.
+    N = 72 and 1029 take the row-store path (N not a multiple of 8)."""
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    ca, sa = _operands(rng, M, K, 127, 127)
+    cb, sb = _operands(rng, N, K, 127, 127)
+    Y = _gemm_bf16(kq, ca, sa, cb, sb)
+    ref = torch.from_numpy(o.gemm_mxfp4(ca, sa, cb, sb).astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(_bf16_bits(Y), _bf16_bits(ref))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (200, 72, 384), (384, 256, 3072), (4608, 3072, 3072)])
+def test_gemm_bf16_matches_fp32_gemm(kq, M, N, K):
+    """Scales 2^-10 .. 2^10: the bf16 output is the fp32 GEMM's output rounded
+    to bf16, bit for bit (same MMAs, same accumulation), and within the fp32
+    accumulation bound plus half a bf16 unit of the fp64 product."""
+    rng = np.random.default_rng(M + 11 * N + K)
+    ca, sa = _operands(rng, M, K, 117, 137)
+    cb, sb = _operands(rng, N, K, 117, 137)
+    Y16 = _gemm_bf16(kq, ca, sa, cb, sb)
+    Y32 = torch.from_numpy(_gemm(kq, ca, sa, cb, sb).astype(np.float32))
+    assert np.array_equal(_bf16_bits(Y16), _bf16_bits(Y32.to(torch.bfloat16)))
+    if M * N <= 1 << 20:
+        ref = o.gemm_mxfp4(ca, sa, cb, sb)
+        tol = (K / 64 + 64) * 2.0 ** -23 * o.gemm_error_scale(ca, sa, cb, sb)
+        err = np.abs(Y16.to(torch.float64).numpy() - ref)
+        assert np.all(err <= tol + 2.0 ** -8 * (np.abs(ref) + tol))
 
 
 @pytest.mark.parametrize("M,d", [(1, 128), (200, 1152), (4608, 3072)])

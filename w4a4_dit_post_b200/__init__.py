@@ -21,7 +21,7 @@ from .build import LIB_PATH
 __all__ = [
     "abi", "kq_quantize", "kq_quantize_sf_tiled", "kq_quantize_centered", "kq_row_sum",
     "kq_quantize_tc", "kq_transform", "sq_quantize", "kq_expand_params",
-    "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4", "kq_gemm_mxfp4_rank1",
+    "kq_fold_weights", "kq_quantize_weights", "kq_sf_tile", "kq_gemm_mxfp4", "kq_gemm_mxfp4_bf16", "kq_gemm_mxfp4_rank1",
     "kq_dequant",
     "kq_device_status",
     "kq_selftest_bounded_wait",
@@ -60,6 +60,8 @@ _SIGNATURES = {
                                    _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "kq_gemm_mxfp4": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _c_void_p,
                              _c_void_p]),
+    "kq_gemm_mxfp4_bf16": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _c_void_p,
+                                  _c_void_p]),
     "kq_dequant": (_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "kq_device_status": (_int, [ctypes.POINTER(ctypes.c_uint32), _int]),
     "kq_selftest_bounded_wait": (_int, [ctypes.c_uint32, _c_void_p]),
@@ -261,9 +263,7 @@ def kq_sf_tile(scales, out=None):
     return out
 
 
-def kq_gemm_mxfp4(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
-    """Y [M, N] fp32 = MXFP4(A) MXFP4(B)^T from codes [M, K/2] / [N, K/2] and
-    scales tiled by kq_sf_tile."""
+def _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled):
     for name, t in (("a_codes", a_codes), ("b_codes", b_codes)):
         _need_cuda(name, t, (torch.uint8,), 2)
     for name, t in (("a_sf_tiled", a_sf_tiled), ("b_sf_tiled", b_sf_tiled)):
@@ -277,9 +277,27 @@ def kq_gemm_mxfp4(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
         if tuple(t.shape) != ((rows + 127) // 128, K // 128, 512):
             raise ValueError(f"{name} has shape {tuple(t.shape)}, expected "
                              f"{((rows + 127) // 128, K // 128, 512)}")
+    return M, N, K
+
+
+def kq_gemm_mxfp4(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
+    """Y [M, N] fp32 = MXFP4(A) MXFP4(B)^T from codes [M, K/2] / [N, K/2] and
+    scales tiled by kq_sf_tile."""
+    M, N, K = _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled)
     Y = _out(Y, (M, N), torch.float32, a_codes, "Y")
     with torch.cuda.device(a_codes.device):
         _check("kq_gemm_mxfp4", abi().kq_gemm_mxfp4(
+            a_codes.data_ptr(), a_sf_tiled.data_ptr(), b_codes.data_ptr(), b_sf_tiled.data_ptr(),
+            M, N, K, Y.data_ptr(), _stream(a_codes)))
+    return Y
+
+
+def kq_gemm_mxfp4_bf16(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
+    """kq_gemm_mxfp4 with Y [M, N] bf16 (each fp32 sum rounded to nearest even)."""
+    M, N, K = _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled)
+    Y = _out(Y, (M, N), torch.bfloat16, a_codes, "Y")
+    with torch.cuda.device(a_codes.device):
+        _check("kq_gemm_mxfp4_bf16", abi().kq_gemm_mxfp4_bf16(
             a_codes.data_ptr(), a_sf_tiled.data_ptr(), b_codes.data_ptr(), b_sf_tiled.data_ptr(),
             M, N, K, Y.data_ptr(), _stream(a_codes)))
     return Y

@@ -29,6 +29,7 @@
 // drains and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -49,6 +50,13 @@ constexpr int kOpBytes = kTile * kKStep / 2;        // 8 KiB of codes per operan
 constexpr int kSfBytes = 512;
 constexpr int kStageBytes = 2 * kOpBytes + 2 * kSfBytes;
 constexpr int kChunkBytes = kTile * 128;           // one 128-row x 32-column fp32 slice of Y
+constexpr int kStagesBf16 = 4;                     // bf16 Y: the whole tile is staged (32 KiB)
+constexpr int kTileBf16Bytes = kTile * kTile * 2;
+
+// Dynamic shared memory of one CTA (stages, Y staging, barriers).
+__host__ __device__ constexpr int smem_bytes(bool bf16) {
+  return 1024 + (bf16 ? kStagesBf16 : kStages) * kStageBytes + (bf16 ? kTileBf16Bytes : kChunkBytes) + 256;
+}
 constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 256;      // 128 accumulator columns + 8 scale columns
 constexpr int kSfaCol = 128, kSfbCol = 132;
@@ -150,7 +158,7 @@ struct GemmArgs {
   const uint8_t* sfa;        // blocked scales of A: [ceil(M/128)][K/128][512]
   const uint8_t* sfb;        // blocked scales of B
   int m_tiles, n_tiles;
-  float* Y;                  // [M][N] fp32
+  void* Y;                   // [M][N] fp32, or bf16 in the bf16 variant
   const float* mu;           // optional rank-1 term: Y += mu wsum^T (mu [M], wsum [N])
   const float* wsum;
   int tma_store;             // 1: Y leaves through shared memory and TMA stores (N % 4 == 0)
@@ -166,20 +174,25 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // lane as soon as the epilogue has read it, so the next tile's loads and MMAs
 // overlap this tile's stores; two CTAs share an SM.  kRank1: the epilogue adds
 // mu[m] * wsum[n] (kq_gemm_mxfp4_rank1); a compile-time switch, so that the
-// plain GEMM's epilogue keeps its registers.
-template <bool kRank1>
+// plain GEMM's epilogue keeps its registers.  kBf16: Y is bf16
+// (kq_gemm_mxfp4_bf16); the epilogue then stages the whole 128 x 128 tile
+// (32 KiB), hands the accumulator back as soon as it has been read, and the
+// tile leaves by two TMA stores while the next tile's MMAs run.
+template <bool kRank1, bool kBf16>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
             const __grid_constant__ CUtensorMap ymap, const GemmArgs args, unsigned int* devstat) {
+  constexpr int kS = kBf16 ? kStagesBf16 : kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* out_chunk = smem + kStages * kStageBytes;               // [128 rows][128 B], 128B swizzle
-  uint64_t* bars = reinterpret_cast<uint64_t*>(out_chunk + kChunkBytes);
-  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kStages]);
-  const uint32_t accf = smem_addr(&bars[2 * kStages]), acce = smem_addr(&bars[2 * kStages + 1]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kStages + 2]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kStages + 3]);
+  // fp32: one [128 rows][128 B] slice; bf16: two [128 rows][128 B] halves of the tile
+  uint8_t* out_chunk = smem + kS * kStageBytes;                    // 128B swizzle
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_chunk + (kBf16 ? kTileBf16Bytes : kChunkBytes));
+  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kS]);
+  const uint32_t accf = smem_addr(&bars[2 * kS]), acce = smem_addr(&bars[2 * kS + 1]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kS + 2]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kS + 3]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KS = args.k_steps;
@@ -193,7 +206,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
     tma_prefetch_desc(&amap);
     tma_prefetch_desc(&bmap);
     if (args.tma_store) tma_prefetch_desc(&ymap);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
@@ -224,8 +237,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
         const uint8_t* sfa_tile = args.sfa + (size_t)m_tile * KS * kSfBytes;
         const uint8_t* sfb_tile = args.sfb + (size_t)n_tile * KS * kSfBytes;
         for (int kt = 0; kt < KS; ++kt, ++seq) {
-          const int s = seq % kStages;
-          if (seq >= kStages && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(seq / kStages - 1) & 1u)) {
+          const int s = seq % kS;
+          if (seq >= kS && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(seq / kS - 1) & 1u)) {
             *abort_flag = 1;
             atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
             break;
@@ -242,9 +255,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
         }
       }
       if (*abort_flag) {
-        const int lo = issued > kStages ? issued - kStages : 0;
+        const int lo = issued > kS ? issued - kS : 0;
         for (int q = lo; q < issued; ++q)
-          (void)mbar_wait_bounded(full0 + 8 * (q % kStages), (uint32_t)(q / kStages) & 1u);
+          (void)mbar_wait_bounded(full0 + 8 * (q % kS), (uint32_t)(q / kS) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -256,8 +269,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
         bool ok = i == 0 || mbar_wait_bounded(acce, (uint32_t)(i - 1) & 1u);
         if (ok) fence_after_sync();
         for (int kt = 0; ok && kt < KS; ++kt, ++seq) {
-          const int s = seq % kStages;
-          ok = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(seq / kStages) & 1u) && !*abort_flag;
+          const int s = seq % kS;
+          ok = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(seq / kS) & 1u) && !*abort_flag;
           if (!ok) break;
           fence_after_sync();
           const uint32_t st = smem_addr(smem + s * kStageBytes);
@@ -293,63 +306,127 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
     }
   } else {
     // epilogue: warps 2..5 -> TMEM lane quarters (warp % 4); thread = one row
-    const int q = warp & 3;
-    const int etid = tid - 64;
-    const int r_local = 32 * q + lane;
-    for (int i = 0; i < my_tiles; ++i) {
-      const int t = (int)blockIdx.x + i * (int)gridDim.x;
-      const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
-      const int row = m_tile * kTile + r_local;
-      const bool ok = mbar_wait_bounded(accf, (uint32_t)i & 1u);
-      if (epi_any(!ok || *abort_flag)) {
-        if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
-      fence_after_sync();
-      const int n0 = n_tile * kTile;
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
-        if constexpr (kRank1) {
-          // the centring variant's removed mean, restored in fp32
-          const float m = row < args.M ? args.mu[row] : 0.0f;
+    if constexpr (kBf16) {
+      const int q = warp & 3;
+      const int etid = tid - 64;
+      const int r_local = 32 * q + lane;
+      for (int i = 0; i < my_tiles; ++i) {
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
+        const int row = m_tile * kTile + r_local;
+        const bool ok = mbar_wait_bounded(accf, (uint32_t)i & 1u);
+        // the previous tile's stores have read the staging buffer
+        if (args.tma_store && etid == 0) bulk_wait_read_all();
+        if (epi_any(!ok || *abort_flag)) {
+          if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        fence_after_sync();
+        const int n0 = n_tile * kTile;
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+          uint32_t w[16];                  // bf16 pairs, even column in the low half
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int col = n0 + 32 * c + k;
-            const float ws = col < args.N ? __ldg(args.wsum + col) : 0.0f;
-            r[k] = __float_as_uint(__fmaf_rn(m, ws, __uint_as_float(r[k])));
+          for (int k = 0; k < 16; ++k) {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+            w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          if (c == kTile / 32 - 1) {
+            // the whole accumulator is in registers or staged: hand it back
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce);
+          }
+          if (args.tma_store) {
+            // half c / 2 of the tile: [128 rows][64 columns = 128 B], 16-byte
+            // chunk j of a row at (j ^ (row % 8)) * 16 (128-byte swizzle)
+            uint8_t* rowp = out_chunk + (c >> 1) * (kTile * 128) + r_local * 128;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int j = (c & 1) * 4 + u;
+              *reinterpret_cast<uint4*>(rowp + ((j ^ (r_local & 7)) << 4)) =
+                  make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+            }
+          } else if (row < args.M) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.Y) + (size_t)row * args.N + n0 + 32 * c;
+            const int n_valid = args.N - (n0 + 32 * c);
+            const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(w);
+            for (int k = 0; k < 32 && k < n_valid; ++k) dst[k] = src[k];
           }
         }
-        if (c == kTile / 32 - 1) {
-          // the whole accumulator is in registers or staged: hand it back
-          fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acce);
-        }
         if (args.tma_store) {
-          // the previous slice's store has read the staging chunk
-          if (etid == 0) bulk_wait_read_all();
-          epi_barrier();
-          uint8_t* rowp = out_chunk + r_local * 128;
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(rowp + ((u ^ (r_local & 7)) << 4)) =
-                make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+          // generic-proxy writes -> visible to the TMA stores, then all warps done
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           epi_barrier();
           if (etid == 0) {
-            tma_store_2d(&ymap, n0 + 32 * c, m_tile * kTile, smem_addr(out_chunk));
+            tma_store_2d(&ymap, n0, m_tile * kTile, smem_addr(out_chunk));
+            tma_store_2d(&ymap, n0 + 64, m_tile * kTile, smem_addr(out_chunk + kTile * 128));
             bulk_commit();
           }
-        } else if (row < args.M) {
-          float* dst = args.Y + (size_t)row * args.N + n0 + 32 * c;
-          const int n_valid = args.N - (n0 + 32 * c);
-          for (int k = 0; k < 32 && k < n_valid; ++k) dst[k] = __uint_as_float(r[k]);
         }
       }
+      if (args.tma_store && etid == 0) bulk_wait_all();
+    } else {
+      const int q = warp & 3;
+      const int etid = tid - 64;
+      const int r_local = 32 * q + lane;
+      for (int i = 0; i < my_tiles; ++i) {
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
+        const int row = m_tile * kTile + r_local;
+        const bool ok = mbar_wait_bounded(accf, (uint32_t)i & 1u);
+        if (epi_any(!ok || *abort_flag)) {
+          if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        fence_after_sync();
+        const int n0 = n_tile * kTile;
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+          if constexpr (kRank1) {
+            // the centring variant's removed mean, restored in fp32
+            const float m = row < args.M ? args.mu[row] : 0.0f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const int col = n0 + 32 * c + k;
+              const float ws = col < args.N ? __ldg(args.wsum + col) : 0.0f;
+              r[k] = __float_as_uint(__fmaf_rn(m, ws, __uint_as_float(r[k])));
+            }
+          }
+          if (c == kTile / 32 - 1) {
+            // the whole accumulator is in registers or staged: hand it back
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce);
+          }
+          if (args.tma_store) {
+            // the previous slice's store has read the staging chunk
+            if (etid == 0) bulk_wait_read_all();
+            epi_barrier();
+            uint8_t* rowp = out_chunk + r_local * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(rowp + ((u ^ (r_local & 7)) << 4)) =
+                  make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            epi_barrier();
+            if (etid == 0) {
+              tma_store_2d(&ymap, n0 + 32 * c, m_tile * kTile, smem_addr(out_chunk));
+              bulk_commit();
+            }
+          } else if (row < args.M) {
+            float* dst = static_cast<float*>(args.Y) + (size_t)row * args.N + n0 + 32 * c;
+            const int n_valid = args.N - (n0 + 32 * c);
+            for (int k = 0; k < 32 && k < n_valid; ++k) dst[k] = __uint_as_float(r[k]);
+          }
+        }
+      }
+      if (args.tma_store && etid == 0) bulk_wait_all();
     }
-    if (args.tma_store && etid == 0) bulk_wait_all();
   }
 
   fence_before_sync();
@@ -416,10 +493,11 @@ constexpr int kMaxDevices = 64;
 
 namespace kq {
 
-// Shared by kq_gemm_mxfp4 (mu = wsum = NULL) and kq_gemm_mxfp4_rank1.
+// Shared by kq_gemm_mxfp4 (mu = wsum = NULL), kq_gemm_mxfp4_rank1 and
+// kq_gemm_mxfp4_bf16 (bf16: Y is bf16, no rank-1 term).
 int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
                 const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, const float* mu,
-                const float* wsum, float* Y, void* stream, const char* fn) {
+                const float* wsum, void* Y, bool bf16, void* stream, const char* fn) {
   if (M < 0 || N < 0 || K <= 0 || K % 128 != 0)
     return kq::fail(KQ_ERR_INVALID_ARG, "%s: need M, N >= 0 and K a positive multiple of 128", fn);
   if (M == 0 || N == 0) return KQ_OK;
@@ -436,31 +514,38 @@ int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return kq::cuda_fail(err, "cudaGetDevice");
   if (dev < 0 || dev >= kq::kMaxDevices) return kq::fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
-  const size_t smem = 1024 + (size_t)kq::gemm::kStages * kq::gemm::kStageBytes + kq::gemm::kChunkBytes + 256;
+  const size_t smem = (size_t)kq::gemm::smem_bytes(bf16);
   static std::once_flag attr_once[kq::kMaxDevices];
   static cudaError_t attr_err[kq::kMaxDevices];
   std::call_once(attr_once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int s32 = kq::gemm::smem_bytes(false), s16 = kq::gemm::smem_bytes(true);
+    attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel<false, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, s32);
     if (attr_err[dev] == cudaSuccess)
-      attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel<true>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel<true, false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, s32);
+    if (attr_err[dev] == cudaSuccess)
+      attr_err[dev] = cudaFuncSetAttribute(kq::gemm::gemm_kernel<false, true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, s16);
   });
   if (attr_err[dev] != cudaSuccess) return kq::cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
 
   CUtensorMap am, bm, ym;
   if (int st = kq::codes_tmap(&am, a_codes, M, K)) return st;
   if (int st = kq::codes_tmap(&bm, b_codes, N, K)) return st;
-  const bool tma_store = (N % 4) == 0;
+  // TMA stores need 16-byte row strides: N a multiple of 4 (fp32) or 8 (bf16)
+  const bool tma_store = (N % (bf16 ? 8 : 4)) == 0;
   memset(&ym, 0, sizeof(ym));
   if (tma_store) {
-    // Y [M][N] fp32; box 32 columns (128 bytes) x 128 rows, 128-byte swizzle
+    // Y [M][N]; box 128 bytes of a row (32 fp32 or 64 bf16 columns) x 128 rows,
+    // 128-byte swizzle
     PFN_cuTensorMapEncodeTiled_v12000 enc = kq::gemm_encoder();
     const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-    const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
-    const cuuint32_t box[2] = {32, (cuuint32_t)kq::gemm::kTile};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * (bf16 ? 2 : 4)};
+    const cuuint32_t box[2] = {bf16 ? 64u : 32u, (cuuint32_t)kq::gemm::kTile};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(&ym, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Y, dims, strides, box, estr,
+    const CUresult r = enc(&ym, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                           2, Y, dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return kq::fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed (CUresult %d)", (int)r);
@@ -495,8 +580,12 @@ int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = mu != nullptr ? cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel<true>, am, bm, ym, args, devstat)
-                      : cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel<false>, am, bm, ym, args, devstat);
+  if (bf16)
+    err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel<false, true>, am, bm, ym, args, devstat);
+  else if (mu != nullptr)
+    err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel<true, false>, am, bm, ym, args, devstat);
+  else
+    err = cudaLaunchKernelEx(&cfg, kq::gemm::gemm_kernel<false, false>, am, bm, ym, args, devstat);
   if (err != cudaSuccess) return kq::cuda_fail(err, "gemm_kernel launch");
   return kq::check_launch("gemm_kernel launch");
 }
@@ -526,8 +615,8 @@ int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void
 
 int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
                   const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, float* Y, void* stream) {
-  return kq::gemm_launch(a_codes, a_sf_tiled, b_codes, b_sf_tiled, M, N, K, nullptr, nullptr, Y, stream,
-                         "kq_gemm_mxfp4");
+  return kq::gemm_launch(a_codes, a_sf_tiled, b_codes, b_sf_tiled, M, N, K, nullptr, nullptr, Y, false,
+                         stream, "kq_gemm_mxfp4");
 }
 
 int kq_gemm_mxfp4_rank1(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
@@ -537,8 +626,15 @@ int kq_gemm_mxfp4_rank1(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_gemm_mxfp4_rank1: NULL mu or wsum");
   if ((mu && !kq::aligned(mu, 4)) || (wsum && !kq::aligned(wsum, 4)))
     return kq::fail(KQ_ERR_ALIGNMENT, "kq_gemm_mxfp4_rank1: mu and wsum must be 4-byte aligned");
-  return kq::gemm_launch(a_codes, a_sf_tiled, b_codes, b_sf_tiled, M, N, K, mu, wsum, Y, stream,
+  return kq::gemm_launch(a_codes, a_sf_tiled, b_codes, b_sf_tiled, M, N, K, mu, wsum, Y, false, stream,
                          "kq_gemm_mxfp4_rank1");
+}
+
+int kq_gemm_mxfp4_bf16(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,
+                       const uint8_t* b_sf_tiled, int64_t M, int64_t N, int64_t K, void* Y,
+                       void* stream) {
+  return kq::gemm_launch(a_codes, a_sf_tiled, b_codes, b_sf_tiled, M, N, K, nullptr, nullptr, Y, true,
+                         stream, "kq_gemm_mxfp4_bf16");
 }
 
 }  // extern "C"
