@@ -58,11 +58,12 @@ def test_quantize_weights_matches_oracle(kq, N, d):
           f"weights {N}x{d}")
 
 
-def test_quantize_weights_equals_quantized_fold(kq):
+@pytest.mark.parametrize("N,d", [(300, 1152), (300, 3072), (7, 1024)])
+def test_quantize_weights_equals_quantized_fold(kq, N, d):
     """The fused kernel encodes exactly what kq_fold_weights writes: the same
     fp32 evaluation, then the activation encoder on it (sq_quantize with unit
-    scales multiplies by 1, exactly)."""
-    N, d = 300, 1152
+    scales multiplies by 1, exactly).  d = 1152 takes the per-block kernel,
+    d = 3072 and 1024 (d / 32 a multiple of 32) the column-stationary one."""
     p = torch.from_numpy(synthetic.make_params(d // 32, 44)).cuda()
     W = torch.from_numpy(synthetic.make_weights(N, d, 8)).cuda()
     c1, s1 = kq.kq_quantize_weights(W, p)
@@ -71,8 +72,8 @@ def test_quantize_weights_equals_quantized_fold(kq):
     assert torch.equal(c1, c2) and torch.equal(s1, s2)
 
 
-def test_quantize_weights_identity_is_plain_mxfp4(kq):
-    N, d = 64, 512
+@pytest.mark.parametrize("N,d", [(64, 512), (64, 2048)])
+def test_quantize_weights_identity_is_plain_mxfp4(kq, N, d):
     W = synthetic.make_weights(N, d, 9)
     p = synthetic.identity_params(d // 32)
     c, s = kq.kq_quantize_weights(torch.from_numpy(W).cuda(), torch.from_numpy(p).cuda())

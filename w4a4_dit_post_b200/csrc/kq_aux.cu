@@ -127,6 +127,58 @@ fold_quant_kernel(const float* __restrict__ W, const float* __restrict__ params,
   }
 }
 
+// The same, column-stationary, when nb is a multiple of 32: warp w keeps the
+// 32-block column group w % n_cg of the weight rows w / n_cg, w / n_cg + rstep,
+// ..., so each lane keeps one block column and builds its five transposed
+// inverse factors once, instead of loading the 15 parameters and dividing for
+// every block.  Loads, shared-memory transpose and stores as fold_quant_kernel.
+__global__ void __launch_bounds__(kAuxThreads)
+fold_quant_cs_kernel(const float* __restrict__ W, const float* __restrict__ params, int N, int nb,
+                     int rstep, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                     unsigned int* devstat) {
+  __shared__ float4 stage[kAuxThreads / 32][32 * 8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4* st = stage[warp];
+  const int n_cg = nb / 32;
+  const int wglob = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (wglob >= rstep * n_cg) return;          // warp-uniform
+  const int cg = wglob % n_cg;
+  const int j = cg * 32 + lane;               // this lane's block column
+  const float* p = params + 15 * j;
+  float4 B[5];
+  bool bad = false;
+#pragma unroll
+  for (int m = 0; m < 5; ++m) {
+    bad |= lu_params_bad(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+    B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+  }
+  if (bad && wglob < n_cg) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
+  for (int r = wglob / n_cg; r < N; r += rstep) {
+    const size_t g0 = (size_t)r * nb + (size_t)cg * 32;
+    const float4* src = reinterpret_cast<const float4*>(W + g0 * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int L = lane + 32 * i;            // 16-byte chunk of the warp's 4 KiB
+      const int b = L >> 3, c = L & 7;
+      st[b * 8 + (c ^ (b & 7))] = src[L];
+    }
+    __syncwarp();
+    float2 v[16];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 t = st[lane * 8 + (q ^ (lane & 7))];
+      v[2 * q] = make_float2(t.x, t.y);
+      v[2 * q + 1] = make_float2(t.z, t.w);
+    }
+    __syncwarp();
+    butterfly32(v, B);
+    uint4 packed;
+    const uint32_t byte = mxfp4_encode32(v, packed);
+    *reinterpret_cast<uint4*>(codes + (g0 + lane) * 16) = packed;
+    scales[g0 + lane] = (uint8_t)byte;
+  }
+}
+
 // out[r] = scale * sum of row r (bf16 or fp32 input, fp32 accumulation):
 // one warp per row, 16-byte loads.
 __global__ void __launch_bounds__(kAuxThreads)
@@ -259,6 +311,21 @@ int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* param
   const int n_blocks = (int)(N * nb);
   unsigned int* devstat = nullptr;
   if (int st = kq::device_status_address(&devstat)) return st;
+  if (nb % 32 == 0) {
+    // column-stationary: a whole number of warps per 32-block column group
+    int sms = 0;
+    if (int st = kq::sm_count(&sms)) return st;
+    const int n_cg = nb / 32;
+    const int64_t warps_want = (int64_t)sms * 8 * (kq::kAuxThreads / 32);
+    int64_t rstep = warps_want / n_cg;
+    if (rstep < 1) rstep = 1;
+    if (rstep > N) rstep = N;
+    const int64_t warps = rstep * n_cg;
+    const int64_t blocks = (warps + kq::kAuxThreads / 32 - 1) / (kq::kAuxThreads / 32);
+    kq::fold_quant_cs_kernel<<<(unsigned)blocks, kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+        W, params, (int)N, nb, (int)rstep, codes, scales, devstat);
+    return kq::check_launch("fold_quant_cs_kernel launch");
+  }
   // one warp per 32 blocks
   const int64_t lanes = (int64_t)((n_blocks + 31) / 32) * 32;
   kq::fold_quant_kernel<<<kq::grid_for((int)lanes), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
