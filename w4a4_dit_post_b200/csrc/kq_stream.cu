@@ -4,8 +4,8 @@
 // Tiling.  An activation [M][d] is viewed as [M rows][nb blocks][32 elements]
 // (rows contiguous, nb = d / 32).  The nb block columns are cut into NC
 // column groups of C consecutive blocks (C = the largest divisor of nb not
-// above 32) and the rows into row tiles of R rows, R = 2 * floor(256 / C).  A
-// tile (R x C blocks, at most 32 KiB of bf16) arrives in shared memory by one
+// above 32) and the rows into row tiles of R rows, R = floor(256 / C).  A
+// tile (R x C blocks, at most 16 KiB of bf16) arrives in shared memory by one
 // 3-D TMA load (box 32 x C x R, 64-byte swizzle for bf16 rows, 128-byte for
 // fp32 rows); the swizzle makes each thread's 16-byte reads of a whole block
 // conflict-free.
@@ -14,12 +14,17 @@
 // column group b % NC for its whole life and walks every (G / NC)-th row
 // tile.  Its transform coefficients therefore cover only C block columns and
 // are built once, in a small shared table.  Thread t owns block column
-// t % C and the row pair (2 (t / C), 2 (t / C) + 1) of every tile: the two
-// rows share their coefficients, so every butterfly operation is one packed
-// f32x2 instruction on (row 0, row 1) with a broadcast coefficient.  The
-// kernel is also compiled with C fixed at 32 (every d that is a multiple of
-// 1024), so that tile height, stage size and the thread's block offsets are
-// constants; per tile a thread then only advances counters and pointers.
+// t % C and row t / C of every tile: one 32-element block, held as 16
+// float2 pairs of adjacent elements.  The first four Kronecker factors pair
+// whole float2s, so their shears are packed f32x2 FMAs with a broadcast
+// coefficient; the fifth pairs the two halves of each float2 (scalar FMAs).
+// One block per thread keeps a thread under 64 registers, so four CTAs (32
+// warps) share an SM; in this latency-bound loop the extra warps hide more
+// than the packed FMAs of a two-row-per-thread layout (126 registers, 16
+// warps per SM) save.  The kernel is also compiled with C fixed at 32 (every
+// d that is a multiple of 1024), so that tile height, stage size and the
+// thread's block offsets are constants; per tile a thread then only advances
+// counters and pointers.
 //
 // Transform.  Each LU factor A = L U (L = [[1,0],[a,1]], U = [[u,b],[0,1/u]])
 // is split as A = S L'' U' with S = diag(u, 1/u), U' = [[1, b/u], [0, 1]] and
@@ -31,7 +36,7 @@
 // sizes of the summed terms are unchanged: D |L''| |U'| = |L| |U| entrywise.
 //
 // Pipeline.  Thread 0 keeps kStages tiles in flight; each stage is guarded by
-// an mbarrier (bounded waits).  After copying its two blocks into registers
+// an mbarrier (bounded waits).  After copying its block into registers
 // a thread joins a CTA barrier, thread 0 reuses the stage for the tile
 // kStages ahead, and the transform, the MXFP4 encoding and the stores
 // overlap the loads in flight.
@@ -51,7 +56,9 @@ namespace kq {
 // module holds its own copy.
 __device__ unsigned int g_devstat = 0;
 
+// 256 threads and at most 64 registers a thread: four CTAs (32 warps) per SM.
 constexpr int kThreads = 256;
+constexpr int kMinBlocks = 4;
 constexpr int kMaxC = 32;
 
 // kKqCentered: kq_quantize_centered (x - mu formed before the transform).
@@ -92,19 +99,19 @@ struct InLayout<4> {                     // fp32: 128-byte blocks, 128B swizzle
   __device__ static int chunk(int b, int q) { return q ^ (b & 7); }
 };
 
-// Coefficient table row per block column (floats).  KroQuant: ten shear
-// coefficients and 32 diagonal entries, each stored twice (the packed pair
-// of a broadcast operand): 84 floats, 21 16-byte units (odd, so 8 threads
-// on consecutive columns hit distinct bank groups).  SmoothQuant: the 32
-// inverse scales, each stored twice, padded to 68 floats (17 units).
+// Coefficient table row per block column (floats).  KroQuant: the ten shear
+// coefficients, each stored twice (the packed pair of a broadcast operand),
+// then the 32 diagonal entries: 52 floats, 13 16-byte units (odd, so 8
+// threads on consecutive columns hit distinct bank groups).  SmoothQuant:
+// the 32 inverse scales padded to 36 floats (9 units).
 template <Op kOp>
 struct Table {
-  static constexpr int kRowFloats = (kOp == Op::kSqQuant) ? 68 : 84;
+  static constexpr int kRowFloats = (kOp == Op::kSqQuant) ? 36 : 52;
 };
 
 template <int kInBytes>
 struct StageCfg {
-  static constexpr int kStages = (kInBytes == 2) ? 3 : 2;
+  static constexpr int kStages = 2;
 };
 
 // Largest divisor of nb that is at most kMaxC.
@@ -120,7 +127,7 @@ inline Geometry make_geometry(int64_t M, int nb) {
   g.nb = nb;
   g.C = choose_C(nb);
   g.NC = nb / g.C;
-  int R = 2 * (kThreads / g.C);
+  int R = kThreads / g.C;
   if (R > 256) R = 256;                  // TMA box dimension limit
   g.R = R;
   g.M = (int)M;
@@ -131,11 +138,11 @@ inline Geometry make_geometry(int64_t M, int nb) {
 }
 
 // Stage size of a tile when the column-group width kC is fixed at compile time
-// (the same formula as make_geometry's: R = 2 * (kThreads / C) rows).
+// (the same formula as make_geometry's: R = kThreads / C rows).
 template <int kInBytes, int kC>
 struct FixedStageBytes {
   static constexpr int value =
-      (2 * (kThreads / kC) * kC * InLayout<kInBytes>::kBlockBytes + 1023) & ~1023;
+      ((kThreads / kC) * kC * InLayout<kInBytes>::kBlockBytes + 1023) & ~1023;
 };
 
 template <int kInBytes, Op kOp>
@@ -145,156 +152,109 @@ inline size_t smem_bytes(const Geometry& g) {
          (size_t)g.C * (Table<kOp>::kRowFloats + 32) * sizeof(float);
 }
 
-// Two blocks (rows 2 rp and 2 rp + 1 of block column c of a tile) from a
-// stage, as 32 packed pairs v[i] = (first row element i, second row element i).
+// One block (row r of block column c of a tile) from a stage: v[k] holds
+// elements (2k, 2k+1).
 template <int kInBytes>
-__device__ __forceinline__ void load_pair(const uint8_t* stage, int C, int rp, int c,
-                                          float2 (&v)[32]) {
+__device__ __forceinline__ void load_row(const uint8_t* stage, int C, int r, int c, float2 (&v)[16]) {
   using L = InLayout<kInBytes>;
-  const int b0 = (2 * rp) * C + c, b1 = b0 + C;
-  const uint8_t* p0 = stage + b0 * L::kBlockBytes;
-  const uint8_t* p1 = stage + b1 * L::kBlockBytes;
+  const int b = r * C + c;
+  const uint8_t* p = stage + b * L::kBlockBytes;
   if constexpr (kInBytes == 2) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 w0 = *reinterpret_cast<const uint4*>(p0 + (L::chunk(b0, q) << 4));
-      const uint4 w1 = *reinterpret_cast<const uint4*>(p1 + (L::chunk(b1, q) << 4));
-      const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w};
-      const uint32_t a1[4] = {w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {  // word e of chunk q holds elements 8q+2e, 8q+2e+1
-        v[8 * q + 2 * e] = make_float2(__uint_as_float(a0[e] << 16), __uint_as_float(a1[e] << 16));
-        v[8 * q + 2 * e + 1] = make_float2(__uint_as_float(a0[e] & 0xffff0000u),
-                                           __uint_as_float(a1[e] & 0xffff0000u));
-      }
+      const uint4 w = *reinterpret_cast<const uint4*>(p + (L::chunk(b, q) << 4));
+      v[4 * q + 0] = bf16x2_to_float2(w.x);
+      v[4 * q + 1] = bf16x2_to_float2(w.y);
+      v[4 * q + 2] = bf16x2_to_float2(w.z);
+      v[4 * q + 3] = bf16x2_to_float2(w.w);
     }
   } else {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const float4 w0 = *reinterpret_cast<const float4*>(p0 + (L::chunk(b0, q) << 4));
-      const float4 w1 = *reinterpret_cast<const float4*>(p1 + (L::chunk(b1, q) << 4));
-      v[4 * q + 0] = make_float2(w0.x, w1.x);
-      v[4 * q + 1] = make_float2(w0.y, w1.y);
-      v[4 * q + 2] = make_float2(w0.z, w1.z);
-      v[4 * q + 3] = make_float2(w0.w, w1.w);
+      const float4 w = *reinterpret_cast<const float4*>(p + (L::chunk(b, q) << 4));
+      v[2 * q] = make_float2(w.x, w.y);
+      v[2 * q + 1] = make_float2(w.z, w.w);
     }
   }
 }
 
-// KroQuant transform of a row pair from one coefficient row.  Row layout:
+// KroQuant transform of one block from its coefficient row.  Row layout:
 // floats [4m .. 4m+3] = (b_m/u_m, b_m/u_m, a_m u_m^2, a_m u_m^2) for m = 0..4,
-// then [20 + 2i], [21 + 2i] = D_i twice for i = 0..31.
-__device__ __forceinline__ void kq_transform_pair(float2 (&v)[32], const float* row) {
+// then [20 + i] = D_i for i = 0..31.  Factor m acts on element-index bit
+// 4 - m, i.e. on bit 3 - m of the pair index k for m < 4 (whole float2s,
+// packed FMA) and inside each float2 for m = 4.
+__device__ __forceinline__ void kq_transform_row(float2 (&v)[16], const float* row) {
   const float4* r4 = reinterpret_cast<const float4*>(row);
 #pragma unroll
-  for (int m = 0; m < 5; ++m) {
-    const int h = 1 << (4 - m);             // factor m acts on element-index bit 4 - m
+  for (int m = 0; m < 4; ++m) {
+    const int h = 1 << (3 - m);
     const float4 sh = r4[m];
     const float2 beta = make_float2(sh.x, sh.y), gamma = make_float2(sh.z, sh.w);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (i & h) continue;
-      v[i] = __ffma2_rn(beta, v[i + h], v[i]);        // U':  lo += (b/u) hi
-      v[i + h] = __ffma2_rn(gamma, v[i], v[i + h]);   // L'':  hi += (a u^2) lo
+    for (int k = 0; k < 16; ++k) {
+      if (k & h) continue;
+      v[k] = __ffma2_rn(beta, v[k + h], v[k]);        // U':  lo += (b/u) hi
+      v[k + h] = __ffma2_rn(gamma, v[k], v[k + h]);   // L'':  hi += (a u^2) lo
+    }
+  }
+  {
+    const float4 sh = r4[4];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      v[k].x = __fmaf_rn(sh.x, v[k].y, v[k].x);
+      v[k].y = __fmaf_rn(sh.z, v[k].x, v[k].y);
     }
   }
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const float4 dd = r4[5 + q];            // (D_2q, D_2q, D_2q+1, D_2q+1)
+  for (int q = 0; q < 8; ++q) {
+    const float4 dd = r4[5 + q];            // D_4q .. D_4q+3
     v[2 * q] = __fmul2_rn(v[2 * q], make_float2(dd.x, dd.y));
     v[2 * q + 1] = __fmul2_rn(v[2 * q + 1], make_float2(dd.z, dd.w));
   }
 }
 
-__device__ __forceinline__ void sq_transform_pair(float2 (&v)[32], const float* row) {
+__device__ __forceinline__ void sq_transform_row(float2 (&v)[16], const float* row) {
   const float4* r4 = reinterpret_cast<const float4*>(row);
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
+  for (int q = 0; q < 8; ++q) {
     const float4 s = r4[q];
     v[2 * q] = __fmul2_rn(v[2 * q], make_float2(s.x, s.y));
     v[2 * q + 1] = __fmul2_rn(v[2 * q + 1], make_float2(s.z, s.w));
   }
 }
 
-template <int kSel>
-__device__ __forceinline__ float lane(const float2& p) {
-  return kSel ? p.y : p.x;
-}
-
-// Largest magnitude of lane kSel (0: first row, 1: second), NaN-propagating.
-template <int kSel>
-__device__ __forceinline__ float lane_absmax(const float2 (&v)[32]) {
-  float m[11];
-#pragma unroll
-  for (int i = 0; i < 10; ++i)
-    m[i] = absmax3(lane<kSel>(v[3 * i]), lane<kSel>(v[3 * i + 1]), lane<kSel>(v[3 * i + 2]));
-  m[10] = absmax2(lane<kSel>(v[30]), lane<kSel>(v[31]));
-  const float q0 = max3(m[0], m[1], m[2]), q1 = max3(m[3], m[4], m[5]);
-  const float q2 = max3(m[6], m[7], m[8]), q3 = max3(m[9], m[10], q0);
-  return max3(q1, q2, q3);
-}
-
-// E2M1 codes of lane kSel: 16 bytes, element 2k in the low nibble of byte k.
-template <int kSel>
-__device__ __forceinline__ uint4 lane_codes(const float2 (&r)[32]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int b = 8 * q;
-    w[q] = e2m1x8(make_float2(lane<kSel>(r[b]), lane<kSel>(r[b + 1])),
-                  make_float2(lane<kSel>(r[b + 2]), lane<kSel>(r[b + 3])),
-                  make_float2(lane<kSel>(r[b + 4]), lane<kSel>(r[b + 5])),
-                  make_float2(lane<kSel>(r[b + 6]), lane<kSel>(r[b + 7])));
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Transform of one row pair of one block column and its output: the
-// transformed values (kq_transform), or the E2M1 codes and E8M0 scale bytes.
-// Rows r0 and r0 + 1 (the second only when `second`), block column jc; g0 =
-// r0 * nb + jc is the flat block index, and cdst, sdst, ydst point at block
-// g0 of codes, scales and y.
+// Transform of one block (row r, block column jc) and its output: the
+// transformed values (kq_transform), or the E2M1 codes and E8M0 scale byte.
+// cdst, sdst and ydst point at the block in codes, scales and y.
 template <Op kOp>
-__device__ __forceinline__ void quantize_pair(float2 (&v)[32], const float* crow, const Geometry& geo,
-                                              int r0, bool second, int jc, uint8_t* cdst,
-                                              uint8_t* sdst, float* ydst, uint8_t* __restrict__ scales) {
-  const int nb = geo.nb;
+__device__ __forceinline__ void quantize_row(float2 (&v)[16], const float* crow, const Geometry& geo,
+                                             int r, int jc, uint8_t* cdst, uint8_t* sdst, float* ydst,
+                                             uint8_t* __restrict__ scales) {
   if constexpr (kOp == Op::kSqQuant) {
-    sq_transform_pair(v, crow);
+    sq_transform_row(v, crow);
   } else {
-    kq_transform_pair(v, crow);
+    kq_transform_row(v, crow);
   }
   if constexpr (kOp == Op::kKqTransform) {
     float4* d0 = reinterpret_cast<float4*>(ydst);
-    float4* d1 = reinterpret_cast<float4*>(ydst + (size_t)nb * 32);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      d0[q] = make_float4(v[4 * q].x, v[4 * q + 1].x, v[4 * q + 2].x, v[4 * q + 3].x);
-      if (second)
-        d1[q] = make_float4(v[4 * q].y, v[4 * q + 1].y, v[4 * q + 2].y, v[4 * q + 3].y);
-    }
+    for (int q = 0; q < 8; ++q) d0[q] = make_float4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
   } else {
-    const uint32_t e0 = e8m0_byte(lane_absmax<0>(v));
-    const uint32_t e1 = e8m0_byte(lane_absmax<1>(v));
-    const float2 sc = make_float2(inv_scale_from_byte(e0), inv_scale_from_byte(e1));
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], sc);
-    *reinterpret_cast<uint4*>(cdst) = lane_codes<0>(v);
+    uint4 out;
+    const uint32_t e = mxfp4_encode32(v, out);
+    *reinterpret_cast<uint4*>(cdst) = out;
     if (geo.sf_tiled) {
-      scales[sf_tiled_offset(r0, jc, nb)] = (uint8_t)e0;
-      if (second) scales[sf_tiled_offset(r0 + 1, jc, nb)] = (uint8_t)e1;
+      scales[sf_tiled_offset(r, jc, geo.nb)] = (uint8_t)e;
     } else {
-      sdst[0] = (uint8_t)e0;
-      if (second) sdst[nb] = (uint8_t)e1;
+      *sdst = (uint8_t)e;
     }
-    if (second) *reinterpret_cast<uint4*>(cdst + (size_t)nb * 16) = lane_codes<1>(v);
   }
 }
 
 // kC: the column-group width when it is fixed at compile time (32, every
 // d that is a multiple of 1024), else 0 and the width comes from geo.
 template <int kInBytes, Op kOp, int kC>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ coef_src,
               const Geometry geo, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
               float* __restrict__ y_out, const float* __restrict__ mu) {
@@ -311,7 +271,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
 
   const int tid = threadIdx.x;
   __builtin_assume(tid < kThreads);
-  const int C = kC ? kC : geo.C, R = kC ? 2 * (kThreads / (kC ? kC : 1)) : geo.R;
+  const int C = kC ? kC : geo.C, R = kC ? (kThreads / (kC ? kC : 1)) : geo.R;
   const int col_group = blockIdx.x % geo.NC;
   const int row_step = gridDim.x / geo.NC;      // CTAs sharing this column group
   const int rt_first = blockIdx.x / geo.NC;
@@ -371,7 +331,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
     __syncthreads();
     for (int i = tid; i < C * 32; i += kThreads) {
       const float sv = stage_in[i];
-      *reinterpret_cast<float2*>(table + (i >> 5) * kRow + 2 * (i & 31)) = make_float2(sv, sv);
+      table[(i >> 5) * kRow + (i & 31)] = sv;
     }
   } else {
     float* prm = table + C * kRow;                      // C * 15 parameters
@@ -396,23 +356,22 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
       float dval = 1.0f;
 #pragma unroll
       for (int m = 0; m < 5; ++m) dval = __fmul_rn(dval, uu[10 * cc + 2 * m + ((e >> (4 - m)) & 1)]);
-      *reinterpret_cast<float2*>(table + cc * kRow + 20 + 2 * e) = make_float2(dval, dval);
+      table[cc * kRow + 20 + e] = dval;
     }
   }
   __syncthreads();
 
-  const int c = tid % C, rp = tid / C;
-  const bool active = rp < R / 2;
+  const int c = tid % C, rr = tid / C;
+  const bool active = rr < R;
   const float* crow = table + c * kRow;
   const int nb = geo.nb;
 
   // Tiles walk the stages in order; the barrier phase flips once per round of
   // kStages tiles (a counter and a flag instead of a division per tile).
-  // Unrolling this loop over the stages made ptxas spill.
   int rt = rt_first;
   uint32_t parity = 0;
-  // this thread's first row, and its output blocks, advanced by a constant per tile
-  int r0 = rt_first * R + 2 * rp;
+  // this thread's row, and its output block, advanced by a constant per tile
+  int r0 = rt_first * R + rr;
   const int r_step = row_step * R;
   const size_t g_first = (size_t)r0 * nb + j0 + c, g_step = (size_t)r_step * nb;
   constexpr bool kCodes = kOp != Op::kKqTransform;   // the other output is NULL
@@ -423,19 +382,18 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
 #pragma unroll 1
     for (int s = 0; s < kStages; ++s, rt += row_step, r0 += r_step) {
       if (rt >= geo.n_row_tiles) return;
-      float2 v[32];
-      // centring variant: this row pair's offsets (read before the wait, so
-      // the load overlaps it)
+      float2 v[16];
+      // centring variant: this row's offset (read before the wait, so the
+      // load overlaps it)
       float2 neg_mu = make_float2(0.0f, 0.0f);
-      if (kOp == Op::kKqCentered && active)
-        neg_mu = make_float2(r0 < geo.M ? -mu[r0] : 0.0f, r0 + 1 < geo.M ? -mu[r0 + 1] : 0.0f);
+      if (kOp == Op::kKqCentered && active && r0 < geo.M) neg_mu = make_float2(-mu[r0], -mu[r0]);
       const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity);
       if (ok) {
         if (active) {
-          load_pair<kInBytes>(smem + s * stage_bytes, C, rp, c, v);
+          load_row<kInBytes>(smem + s * stage_bytes, C, rr, c, v);
           if constexpr (kOp == Op::kKqCentered) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __fadd2_rn(v[i], neg_mu);
+            for (int i = 0; i < 16; ++i) v[i] = __fadd2_rn(v[i], neg_mu);
           }
         }
       } else {
@@ -462,8 +420,8 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
           tma_load_3d(smem_addr(smem + s * stage_bytes), &tmap, 0, j0, nrt * R, smem_addr(&bars[s]));
         }
       }
-      if (active && r0 < geo.M)                   // rows r0 and r0 + 1
-        quantize_pair<kOp>(v, crow, geo, r0, r0 + 1 < geo.M, j0 + c, cdst, sdst, ydst, scales);
+      if (active && r0 < geo.M)
+        quantize_row<kOp>(v, crow, geo, r0, j0 + c, cdst, sdst, ydst, scales);
       if constexpr (kCodes) {
         cdst += g_step * 16;
         sdst += g_step;
