@@ -7,7 +7,6 @@
 //  * the MXFP4 block encoder (amax, E8M0 byte, E2M1 nibbles).
 #pragma once
 
-#include <cuda_fp4.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -235,15 +234,23 @@ __device__ __forceinline__ float inv_scale_from_byte(uint32_t byte) {
 }
 
 // Four pairs -> 8 E2M1 nibbles in one word; element 2i of the pair list lands
-// in nibble 2i (low nibble first).  The conversion is CUDA's own
-// __nv_cvt_float2_to_fp4x2 (round to nearest even, saturating to +-6), which
-// puts x.x in the low nibble of its byte.
+// in nibble 2i (low nibble first).  Each pair goes through the PTX conversion
+// cvt.rn.satfinite.e2m1x2.f32 (round to nearest even, saturating to +-6),
+// whose first source lands in the upper nibble of the byte, so a pair (x, y)
+// is passed as (y, x).  The four bytes are packed by a vector mov (byte 0
+// first): ptxas then keeps them in byte lanes instead of widening each one to
+// a word and shifting it into place.
 __device__ __forceinline__ uint32_t e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3) {
-  const uint32_t b0 = __nv_cvt_float2_to_fp4x2(p0, __NV_E2M1, cudaRoundNearest);
-  const uint32_t b1 = __nv_cvt_float2_to_fp4x2(p1, __NV_E2M1, cudaRoundNearest);
-  const uint32_t b2 = __nv_cvt_float2_to_fp4x2(p2, __NV_E2M1, cudaRoundNearest);
-  const uint32_t b3 = __nv_cvt_float2_to_fp4x2(p3, __NV_E2M1, cudaRoundNearest);
-  return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+  uint32_t w;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+      "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+      : "=r"(w)
+      : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+  return w;
 }
 
 // Encode 32 values: returns the scale byte and writes 16 code bytes to `out`.

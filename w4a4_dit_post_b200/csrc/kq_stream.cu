@@ -56,9 +56,7 @@ namespace kq {
 // module holds its own copy.
 __device__ unsigned int g_devstat = 0;
 
-// 256 threads and at most 64 registers a thread: four CTAs (32 warps) per SM.
 constexpr int kThreads = 256;
-constexpr int kMinBlocks = 4;
 constexpr int kMaxC = 32;
 
 // kKqCentered: kq_quantize_centered (x - mu formed before the transform).
@@ -108,6 +106,15 @@ template <Op kOp>
 struct Table {
   static constexpr int kRowFloats = (kOp == Op::kSqQuant) ? 36 : 52;
 };
+
+// CTAs per SM that the register budget is sized for.  bf16 input: four
+// (64 registers a thread, 32 warps per SM; four CTAs' shared memory fits).
+// kq_transform's fp32 stores need more registers than that: three (85).
+// fp32 input: only two CTAs' shared memory fits, so two (128 registers).
+template <int kInBytes, Op kOp>
+constexpr int min_blocks_per_sm() {
+  return kInBytes == 4 ? 2 : (kOp == Op::kKqTransform ? 3 : 4);
+}
 
 template <int kInBytes>
 struct StageCfg {
@@ -254,7 +261,7 @@ __device__ __forceinline__ void quantize_row(float2 (&v)[16], const float* crow,
 // kC: the column-group width when it is fixed at compile time (32, every
 // d that is a multiple of 1024), else 0 and the width comes from geo.
 template <int kInBytes, Op kOp, int kC>
-__global__ void __launch_bounds__(kThreads, kMinBlocks)
+__global__ void __launch_bounds__(kThreads, (min_blocks_per_sm<kInBytes, kOp>()))
 stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict__ coef_src,
               const Geometry geo, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
               float* __restrict__ y_out, const float* __restrict__ mu) {
