@@ -139,7 +139,7 @@ def test_gemm_bf16_matches_fp32_gemm(kq, M, N, K):
         assert np.all(err <= tol + 2.0 ** -8 * (np.abs(ref) + tol))
 
 
-@pytest.mark.parametrize("M,d", [(1, 128), (200, 1152), (4608, 3072)])
+@pytest.mark.parametrize("M,d", [(1, 128), (200, 1152), (1031, 3072), (4608, 3072)])
 def test_quantize_with_tiled_scales(kq, M, d):
     """kq_quantize_sf_tiled writes the codes of kq_quantize and the scale
     blocks kq_sf_tile makes from kq_quantize's scales (rows past M untouched)."""

@@ -45,7 +45,10 @@ def check(rep, label):
 # ---------------------------------------------------------------------------
 # small shapes, every element
 # ---------------------------------------------------------------------------
-SMALL = [(1, 32), (3, 64), (7, 96), (129, 96), (256, 1152), (300, 160), (1031, 224)]
+# (13, 3072) and (1031, 1024) run the kernel compiled for 32-block column groups
+# on a row count that ends inside a tile (8 rows per tile)
+SMALL = [(1, 32), (3, 64), (7, 96), (129, 96), (256, 1152), (300, 160), (1031, 224), (13, 3072),
+         (1031, 1024)]
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
