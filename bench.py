@@ -249,7 +249,7 @@ def weight_bytes(N: int, d: int) -> float:
     return N * d * (4 + 0.5 + 1 / 32) + (d // 32) * 60
 
 
-def time_weight_side(kq, device, stream, K: int, W: int) -> dict:
+def time_weight_side(kq, device, stream, K: int, W: int, shapes=WEIGHT_SHAPES) -> dict:
     """kq_quantize_weights on the FLUX.1-schnell layer weight shapes: mean
     device time of K back-to-back launches (each shape's weights are 38-151
     MB, so a ring of 2 sets already exceeds L2)."""
@@ -257,7 +257,7 @@ def time_weight_side(kq, device, stream, K: int, W: int) -> dict:
     lib = kq.abi()
     peak, _ = hbm_peak()
     out = {"kernel": "kq_quantize_weights (fold W T^-1 + MXFP4, fp32 in)", "shapes": {}}
-    for N, d in WEIGHT_SHAPES:
+    for N, d in shapes:
         sets = []
         for r in range(2):
             Wt = torch.from_numpy(synthetic.make_weights(N, d, 20 + r)).to(device)
@@ -519,6 +519,15 @@ def run_kroquant(args) -> int:
         if rank == 0:
             print(json.dumps({"profile": f"kq_gemm_mxfp4 and kq_gemm_mxfp4_bf16 {M}x{N}x{Kd}", "launches": 2 * (W + K),
                               **r["shapes"][f"{M}x{N}x{Kd}"],
+                              "device_status": kq.kq_device_status(device)}), flush=True)
+        return 0
+    if args.profile == "weights":
+        # only kq_quantize_weights launches on the FLUX MLP-in weight (for ncu captures)
+        N, d = WEIGHT_SHAPES[1]
+        r = time_weight_side(kq, device, stream, K, W, shapes=[(N, d)])
+        if rank == 0:
+            print(json.dumps({"profile": f"kq_quantize_weights {N}x{d}", "launches": W + K,
+                              **r["shapes"][f"{N}x{d}"],
                               "device_status": kq.kq_device_status(device)}), flush=True)
         return 0
     if args.profile:
@@ -795,10 +804,12 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["kroquant", "reference"], default="kroquant")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", nargs="?", const="kq", choices=["kq", "tc", "gemm"], default=None,
+    ap.add_argument("--profile", nargs="?", const="kq", choices=["kq", "tc", "gemm", "weights"],
+                    default=None,
                     help="run only the kq_quantize (kq), kq_quantize_tc (tc) launches of the largest "
-                         "shape, or the kq_gemm_mxfp4 launches of the first layer shape (gemm), "
-                         "for ncu captures")
+                         "shape, the kq_gemm_mxfp4 launches of the first layer shape (gemm), or the "
+                         "kq_quantize_weights launches of the 12288 x 3072 weight (weights), for ncu "
+                         "captures")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     _, world, _ = dist_env()
