@@ -23,7 +23,7 @@ Sources (cited by page title and section):
   largest exponent (2 for E2M1); elements are rounded to nearest-even and
   saturated to the largest finite magnitude (6).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * factor form: A = L U with L = [[1, 0], [a, 1]] and U = [[u, b], [0, 1/u]],
   three parameters (a, b, u) per factor, fifteen per block;
