@@ -47,7 +47,10 @@ WORKLOAD = "flux"
 BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
 PARAM_BYTES_PER_BLOCK_COL = 15 * 4
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 7700.0      # B200 HBM3e, NVIDIA's HGX figure (8 TB/s for DGX)
 RING_FACTOR_L2 = 4.0
+LAUNCHES_PER_REP = 200        # per-launch numbers: median of REPS bursts of this many launches
+REPS = 5
 PAGES_CONTEXT = ("the pages report the KroQuant quantizer kernel up to 14% faster than "
                  "the SmoothQuant kernel on AMD MI350 (relative only; shapes not given)")
 
@@ -79,6 +82,22 @@ def ring_depth(w, l2_bytes: int) -> int:
     including back-to-back launches of one shape, reads cold data)."""
     per_launch = w.M * w.d * (2 + 0.5 + 1 / 32)
     return max(2, int(math.ceil(RING_FACTOR_L2 * l2_bytes / per_launch)))
+
+
+def step_config(world: int) -> dict:
+    """The workload description both arms print (identical for the GPU arm
+    and the reference arm)."""
+    ws = step_workloads(0)
+    return {
+        "workload": "FLUX.1-schnell-shaped linear-layer inputs: M=4608 tokens x d in "
+                    "{3072, 12288}, bf16 in -> MXFP4 (E2M1 codes + E8M0 scales) out; "
+                    "one kq_quantize launch per shape per step",
+        "M_per_rank": ws[0].M,
+        "d": [w.d for w in ws],
+        "l2": f"inputs larger than L2: each shape cycles through its own ring of distinct "
+              f"input/output sets, each ring more than {RING_FACTOR_L2:.0f} x the L2 size",
+        "parallelism": f"replicas x{world} (token rows per rank, no collective)",
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -235,6 +254,136 @@ def ncu_traffic():
         return None, "ncu summary predates the current kernel sources"
     except Exception as e:
         return None, f"no ncu summary ({type(e).__name__})"
+
+
+# ---------------------------------------------------------------------------
+# per-launch timing: REPS bursts of LAUNCHES_PER_REP back-to-back launches
+# ---------------------------------------------------------------------------
+def launch_times_us(launch, n: int = LAUNCHES_PER_REP, reps: int = REPS, warm: int = 10):
+    """Device time per launch of `launch(k, stream_ptr)` (k = the launch's
+    index, for cycling an input ring).  The n launches of a burst are
+    captured once in a CUDA graph and the graph is replayed `reps` times
+    between two CUDA events each, so the host's launch rate never limits the
+    short launches; returns (median, list) of the per-launch times in us."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for k in range(warm):
+            launch(k, side.cuda_stream)
+    side.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        cap = torch.cuda.current_stream().cuda_stream
+        for k in range(n):
+            launch(k, cap)
+    times = []
+    with torch.cuda.stream(side):
+        g.replay()                      # the first replay uploads the graph
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(side)
+            g.replay()
+            e1.record(side)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3 / n)
+    del g
+    torch.cuda.synchronize()
+    return statistics.median(times), times
+
+
+def device_rows(w, device, max_host_rows: int = 4096):
+    """The workload's activations on the device.  Up to max_host_rows rows
+    come from the seeded generator; larger M repeats that block of rows (the
+    kernels' cost does not depend on the values, and generating 805 M
+    elements on the host would take minutes)."""
+    import torch
+    rows = np.arange(min(w.M, max_host_rows))
+    raw = synthetic.make_activations(w, rows)
+    if w.dtype == "bf16":
+        blk = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16).to(device)
+    else:
+        blk = torch.from_numpy(raw).to(device)
+    if w.M == rows.size:
+        return blk, raw
+    reps = (w.M + rows.size - 1) // rows.size
+    return blk.repeat(reps, 1)[:w.M].contiguous(), raw
+
+
+def ring_of(x0, n_slots: int, out_shapes):
+    """n_slots distinct (input, outputs...) sets: the input rolled by a
+    different row offset in each, fresh outputs."""
+    import torch
+    slots = []
+    for r in range(n_slots):
+        x = x0 if r == 0 else torch.roll(x0, shifts=r * 997, dims=0).contiguous()
+        slots.append((x,) + tuple(torch.empty(sh, dtype=dt, device=x0.device) for sh, dt in out_shapes))
+    return slots
+
+
+def time_per_config(kq, device, l2: int, names=("tiny", "pixart", "sana", "flux", "sweep")) -> dict:
+    """kq_quantize and sq_quantize on every BASELINE workload shape, and
+    kq_fold_weights on d x d weights for the sweep's widths: median
+    per-launch device time of REPS bursts of LAUNCHES_PER_REP launches over
+    an input ring larger than RING_FACTOR_L2 x L2."""
+    import torch
+    lib = kq.abi()
+    peak, _ = hbm_peak()
+    out = {"timing": f"median of {REPS} CUDA-graph replays of {LAUNCHES_PER_REP} back-to-back "
+                     f"launches, each launch on its own ring slot (rings > {RING_FACTOR_L2:.0f} x L2)",
+           "peak_gbs": peak, "shapes": {}, "fold_weights": {}}
+    for w in synthetic.workloads(names):
+        dt = kq.KQ_DTYPE_BF16 if w.dtype == "bf16" else kq.KQ_DTYPE_F32
+        x0, raw = device_rows(w, device)
+        p = torch.from_numpy(synthetic.make_params(w.nb, w.seed)).to(device)
+        xs = synthetic.f32_from_bf16_bits(raw) if w.dtype == "bf16" else raw
+        inv_s = torch.from_numpy(synthetic.smoothquant_inv_scales(xs[:: max(1, xs.shape[0] // 1024)])).to(device)
+        per = w.M * w.d * ((2 if w.dtype == "bf16" else 4) + 0.5 + 1 / 32)
+        n_slots = max(2, int(math.ceil(RING_FACTOR_L2 * l2 / per)))
+        slots = ring_of(x0, n_slots, [((w.M, w.d // 2), torch.uint8), ((w.M, w.d // 32), torch.uint8)])
+        ptr = [(x.data_ptr(), c.data_ptr(), sc.data_ptr()) for x, c, sc in slots]
+        row = {}
+        for tag, fn, coef in (("kq", lib.kq_quantize, p), ("sq", lib.sq_quantize, inv_s)):
+            def go(k, sp, fn=fn, coef=coef):
+                xp, cp, spp = ptr[k % len(ptr)]
+                st = fn(xp, dt, w.M, w.d, coef.data_ptr(), cp, spp, sp)
+                if st != 0:
+                    raise RuntimeError(lib.kq_last_error().decode())
+            us, _ = launch_times_us(go)
+            bts = algorithmic_bytes(w.M, w.d) + (w.M * w.d * 2 if w.dtype == "f32" else 0)
+            if tag == "sq":
+                bts += w.d * 4 - (w.d // 32) * PARAM_BYTES_PER_BLOCK_COL
+            gbs = bts / (us * 1e-6) / 1e9
+            row.update({f"{tag}_us": round(us, 2), f"{tag}_gbs": round(gbs, 1),
+                        f"{tag}_frac": round(gbs / peak, 4)})
+        row["kq_over_sq_time"] = round(row["kq_us"] / row["sq_us"], 4)
+        row["ring"] = n_slots
+        out["shapes"][w.key] = row
+        del slots, x0, ptr
+        torch.cuda.empty_cache()
+    for d in sorted({w.d for w in synthetic.workloads(["sweep"])}):
+        Wt = torch.from_numpy(synthetic.make_weights(min(d, 4096), d, 90)).to(device)
+        W0 = Wt.repeat((d + Wt.shape[0] - 1) // Wt.shape[0], 1)[:d].contiguous()
+        p = torch.from_numpy(synthetic.make_params(d // 32, 91)).to(device)
+        per = d * d * 8.0
+        n_slots = max(2, int(math.ceil(RING_FACTOR_L2 * l2 / per)))
+        slots = ring_of(W0, n_slots, [((d, d), torch.float32)])
+        ptr = [(a.data_ptr(), b.data_ptr()) for a, b in slots]
+
+        def go(k, sp):
+            a, b = ptr[k % len(ptr)]
+            st = lib.kq_fold_weights(a, d, d, p.data_ptr(), b, sp)
+            if st != 0:
+                raise RuntimeError(lib.kq_last_error().decode())
+        us, _ = launch_times_us(go, n=min(LAUNCHES_PER_REP, 50))
+        bts = d * d * 8.0 + (d // 32) * PARAM_BYTES_PER_BLOCK_COL
+        gbs = bts / (us * 1e-6) / 1e9
+        out["fold_weights"][f"{d}x{d}"] = {"us": round(us, 2), "gbs": round(gbs, 1),
+                                          "frac": round(gbs / peak, 4), "ring": n_slots}
+        del slots, W0, Wt, ptr
+        torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -566,9 +715,27 @@ def run_kroquant(args) -> int:
     sampler.stop()
     clocks = sampler.summary(t0, t1, t2)
     ms_sq, _, _ = timed_steps("sq", K, W)
-    launch_kq = [timed_burst(i, "kq", K, W) for i in range(len(rings))]
-    launch_sq = [timed_burst(i, "sq", K, W) for i in range(len(rings))]
-    launch_tc = timed_burst(dominant, "tc", K, W)
+
+    def graph_launch(i, fn):
+        """Median per-launch time (ms) of shape i, REPS graph replays of
+        LAUNCHES_PER_REP launches through the C ABI."""
+        w = rings[i][0]
+        coef = coef_ptr[i][1 if fn == "sq" else 0]
+
+        def go(k, sp):
+            xp, cp, spp = ptrs[i][k % len(ptrs[i])]
+            st = abi_fn[fn](xp, kq.KQ_DTYPE_BF16, w.M, w.d, coef, cp, spp, sp)
+            if st != 0:
+                raise RuntimeError(f"{fn} launch failed: {lib.kq_last_error().decode()}")
+        med, reps = launch_times_us(go)
+        return med * 1e-3, [round(r, 2) for r in reps]
+
+    launch_kq, reps_kq = zip(*[graph_launch(i, "kq") for i in range(len(rings))])
+    launch_sq, reps_sq = zip(*[graph_launch(i, "sq") for i in range(len(rings))])
+    launch_tc, _ = graph_launch(dominant, "tc")
+    # the same dominant launches issued one by one from the host (no graph), as a cross-check
+    direct_kq = statistics.median(timed_burst(dominant, "kq", LAUNCHES_PER_REP, W) for _ in range(REPS))
+    per_config = time_per_config(kq, device, l2)
     weight_side = time_weight_side(kq, device, stream, K, W)
     w4a4_gemm = time_gemm(kq, device, stream, K, W)
     w4a4_layer = time_layer(kq, device, stream, K, W)
@@ -635,12 +802,16 @@ def run_kroquant(args) -> int:
         per_shape = {}
         for i, w in enumerate(ws):
             bts = algorithmic_bytes(w.M, w.d)
+            sq_bts = bts + w.d * 4 - (w.d // 32) * PARAM_BYTES_PER_BLOCK_COL
             per_shape[f"{w.M}x{w.d}"] = {
                 "kq_us": round(launch_kq[i] * 1e3, 2),
+                "kq_us_reps": reps_kq[i],
                 "kq_gbs": round(bts / (launch_kq[i] * 1e-3) / 1e9, 1),
                 "kq_frac_of_peak": round(bts / (launch_kq[i] * 1e-3) / 1e9 / peak, 4),
                 "sq_us": round(launch_sq[i] * 1e3, 2),
-                "sq_gbs": round(bts / (launch_sq[i] * 1e-3) / 1e9, 1),
+                "sq_us_reps": reps_sq[i],
+                "sq_gbs": round(sq_bts / (launch_sq[i] * 1e-3) / 1e9, 1),
+                "sq_frac_of_peak": round(sq_bts / (launch_sq[i] * 1e-3) / 1e9 / peak, 4),
             }
         line = {
             "metric": METRIC,
@@ -656,19 +827,9 @@ def run_kroquant(args) -> int:
             "dtype": "f32",
             "data": "synthetic (seeded FLUX.1-schnell-shaped activations: N(0,1), 1% outlier "
                     "channels x100, per-token mean N(0,4); random LU parameters)",
-            "config": {
-                "workload": "FLUX.1-schnell-shaped linear-layer inputs: M=4608 tokens x d in "
-                            "{3072, 12288}, bf16 in -> MXFP4 (E2M1 codes + E8M0 scales) out; "
-                            "one kq_quantize launch per shape per step",
-                "M_per_rank": ws[0].M,
-                "d": [w.d for w in ws],
-                "l2": "inputs larger than L2: each shape cycles through its own ring of "
-                      + ", ".join(f"{r} (d={w.d}, {r * algorithmic_bytes(w.M, w.d) / 1e6:.0f} MB)"
-                                  for r, w in zip(Rs, ws))
-                      + f" distinct input/output sets, each ring > {RING_FACTOR_L2:.0f} x L2 "
-                        f"({l2 / 2 ** 20:.0f} MiB)",
-                "parallelism": f"replicas x{world} (token rows per rank, no collective)",
-            },
+            "config": step_config(world),
+            "rings": ", ".join(f"{r} sets (d={w.d}, {r * algorithmic_bytes(w.M, w.d) / 1e6:.0f} MB)"
+                               for r, w in zip(Rs, ws)) + f"; L2 {l2 / 2 ** 20:.0f} MiB",
             "gpu_launches": K * len(ws),
             "roofline": {
                 "bound": "hbm",
@@ -679,7 +840,14 @@ def run_kroquant(args) -> int:
                 "frac": round(achieved / peak, 4),
                 "traffic": traffic,
                 "algorithmic_bytes_per_launch": dom_bytes,
-                "timing": "mean of K back-to-back launches of this shape between two CUDA events",
+                "timing": f"median of {REPS} bursts of {LAUNCHES_PER_REP} back-to-back launches of this "
+                          f"shape (a CUDA graph of the C-ABI calls, replayed between two CUDA events "
+                          f"on the launching stream), each launch on its own ring slot",
+                "us_per_launch": round(launch_kq[dominant] * 1e3, 2),
+                "us_per_launch_reps": reps_kq[dominant],
+                "us_per_launch_direct": round(direct_kq * 1e3, 2),
+                "frac_of_nominal_hbm": round(achieved / NOMINAL_HBM_GBS, 4),
+                "nominal_hbm_gbs": NOMINAL_HBM_GBS,
                 "peak_source": peak_src,
                 "traffic_source": traffic_src,
             },
@@ -696,6 +864,7 @@ def run_kroquant(args) -> int:
                 "gbs": round(dom_bytes / (launch_tc * 1e-3) / 1e9, 1),
                 "frac_of_peak": round(dom_bytes / (launch_tc * 1e-3) / 1e9 / peak, 4),
             },
+            "per_config": per_config,
             "weight_side": weight_side,
             "w4a4_gemm": w4a4_gemm,
             "w4a4_layer": w4a4_layer,
@@ -748,33 +917,124 @@ def _single_thread():
         return contextlib.nullcontext()
 
 
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_worker(rows_by_shape, steps, barrier, queue):
+    """One process of the all-core oracle run: its own token rows of each
+    FLUX shape, generated before the first step; every step starts on a
+    barrier shared by all workers and times one oracle pass over the rows."""
+    os.environ["OMP_NUM_THREADS"] = "1"
+    with _single_thread():
+        import oracle.kq_oracle as o
+        ws = step_workloads(0)
+        data = []
+        for w, (r0, r1) in zip(ws, rows_by_shape):
+            rows = np.arange(r0, r1)
+            x = synthetic.f32_from_bf16_bits(synthetic.make_activations(w, rows)).astype(np.float64)
+            data.append((x, synthetic.make_params(w.nb, w.seed), rows.size * w.d * BYTES_PER_ELEM))
+        for step in range(steps):
+            barrier.wait(timeout=600)
+            t0 = time.perf_counter()
+            nbytes = 0.0
+            for x, p, b in data:
+                if x.shape[0]:
+                    o.kq_quantize(x, p)
+                    nbytes += b
+            queue.put((step, t0, time.perf_counter(), nbytes))
+
+
+def oracle_all_cores(rows_per_worker: int, steps: int, workers: int | None = None):
+    """The oracle on every host core at once: one spawned process per core,
+    each quantizing its own rows_per_worker tokens of both FLUX shapes per
+    step.  Returns (workers, [(seconds, bytes) per step]); a step's time runs
+    from the first worker's start to the last worker's end."""
+    import multiprocessing as mp
+    ws = step_workloads(0)
+    n = workers or host_cores()
+    n = max(1, min(n, ws[0].M // max(1, rows_per_worker)))
+    ctx = mp.get_context("spawn")
+    barrier = ctx.Barrier(n)
+    queue = ctx.Queue()
+    procs = []
+    for i in range(n):
+        rb = [(i * rows_per_worker, min(w.M, (i + 1) * rows_per_worker)) for w in ws]
+        pr = ctx.Process(target=_oracle_worker, args=(rb, steps, barrier, queue), daemon=True)
+        pr.start()
+        procs.append(pr)
+    res = [[] for _ in range(steps)]
+    for _ in range(n * steps):
+        step, t0, t1, b = queue.get(timeout=1800)
+        res[step].append((t0, t1, b))
+    for pr in procs:
+        pr.join(timeout=60)
+    out = []
+    for r in res:
+        out.append((max(t1 for _, t1, _ in r) - min(t0 for t0, _, _ in r), sum(b for _, _, b in r)
+                    + sum((w.d // 32) * PARAM_BYTES_PER_BLOCK_COL for w in ws)))
+    return n, out
+
+
 def cpu_baseline(seconds: float = 15.0) -> dict:
+    """The oracle as it stands on the host: one thread on a bounded sample
+    of tokens, then every core at once (one process per core), about
+    `seconds` of CPU work each way."""
     ws = step_workloads(0)
     with _single_thread():
         s, b = _oracle_sample(ws, 16)                      # calibrate
-        rows = int(max(16, min(4608, 16 * seconds / max(s, 1e-3))))
+        rows = int(max(16, min(4608, 16 * seconds / 2 / max(s, 1e-3))))
         s, b = _oracle_sample(ws, rows)
-    return {"value": round(b / s / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} of 4608 tokens of each FLUX shape (3072, 12288), fp64 NumPy "
-                      f"oracle, one thread, {s:.1f} s"}
+    single = b / s / 1e9
+    cores = host_cores()
+    per_worker = int(max(8, min(4608 // cores, rows)))
+    try:
+        n, steps = oracle_all_cores(per_worker, 1, cores)
+        secs, nb = steps[0]
+        allc = {"value": round(nb / secs / 1e9, 6), "cores": n,
+                "sample": f"{per_worker} tokens of each FLUX shape per process, {n} processes, "
+                          f"{secs:.1f} s"}
+    except Exception as e:          # the single-thread figure still stands
+        allc = {"value": None, "cores": 0, "sample": f"all-core run failed: {type(e).__name__}: {e}"}
+    best = allc if allc["value"] else {"value": round(single, 6), "cores": 1}
+    return {"value": best["value"], "unit": UNIT, "cores": best["cores"], "kind": "oracle",
+            "sample": f"fp64 NumPy oracle on the FLUX shapes (3072, 12288): {allc['sample']}; "
+                      f"single thread on the first {rows} tokens of each shape, {s:.1f} s",
+            "single_thread": {"value": round(single, 6), "cores": 1},
+            "all_cores": allc, "cpu_model": cpu_model(), "host_cores": cores}
 
 
 def run_reference(args) -> int:
+    """The reference arm: the CPU oracle on all host cores, each step a
+    bounded sample of the FLUX workload's tokens (rank 0 only)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     ws = step_workloads(0)
+    cores = host_cores()
     with _single_thread():
-        s, _ = _oracle_sample(ws, 8)
-        budget = 150.0 / max(1, args.steps + args.warmup)   # whole run within a few minutes
-        rows = int(max(8, min(4608, 8 * budget / max(s, 1e-3))))
-        for _ in range(args.warmup):
-            _oracle_sample(ws, rows)
-        tot_s, tot_b = 0.0, 0.0
-        for _ in range(args.steps):
-            s, b = _oracle_sample(ws, rows)
-            tot_s += s
-            tot_b += b
+        s, _ = _oracle_sample(ws, 8)                       # seconds for 8 tokens, one core
+    budget = 120.0 / max(1, args.steps + args.warmup)      # whole run within a few minutes
+    per_worker = int(max(8, min(4608 // cores, 8 * budget / max(s, 1e-3))))
+    n, steps = oracle_all_cores(per_worker, args.warmup + args.steps, cores)
+    timed = steps[args.warmup:]
+    tot_s = sum(t for t, _ in timed)
+    tot_b = sum(b for _, b in timed)
     value = tot_b / tot_s / 1e9
     line = {
         "impl": "reference",
@@ -782,13 +1042,14 @@ def run_reference(args) -> int:
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(tot_s / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded FLUX.1-schnell-shaped activations)",
-        "config": {"workload": "FLUX.1-schnell-shaped linear-layer inputs: M=4608 tokens x d in "
-                               "{3072, 12288}, bf16 in -> MXFP4 out; each step a bounded sample "
-                               f"of {rows} tokens per shape",
-                   "M_per_rank": 4608, "d": [w.d for w in ws]},
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"first {rows} tokens of each FLUX shape per step"},
+        "data": "synthetic (seeded FLUX.1-schnell-shaped activations: N(0,1), 1% outlier "
+                "channels x100, per-token mean N(0,4); random LU parameters)",
+        "config": step_config(world),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": n, "kind": "oracle",
+                         "sample": f"each step: {per_worker} tokens of each FLUX shape per process, "
+                                   f"{n} processes (one per host core) on {n * per_worker} of the "
+                                   f"4608 tokens",
+                         "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

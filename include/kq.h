@@ -140,7 +140,10 @@ int kq_row_sum(const void* x, int x_dtype, int64_t M, int64_t d, float scale, fl
                void* stream);
 
 /*
- * kq_transform -- the transform stage alone: y = blockdiag(T_j) x in fp32.
+ * kq_transform -- the transform stage alone: y = blockdiag(T_j) x in fp32
+ * (the abstract: an invertible linear transform applied to the activations,
+ * block by block over 32 channels; research summary, method paragraph: each
+ * block's matrix is the Kronecker product of five 2x2 LU factors).
  * Same arguments and limits as kq_quantize; y [M][d] fp32, 16-byte aligned.
  * It runs the same transform code as kq_quantize, so kq_quantize's codes are
  * the MXFP4 encoding of exactly these values.
@@ -159,7 +162,10 @@ int sq_quantize(const void* x, int x_dtype, int64_t M, int64_t d,
                 void* stream);
 
 /*
- * kq_expand_params -- the dense blocks of the transform.
+ * kq_expand_params -- the dense blocks of the transform (research summary,
+ * method paragraph: each 32-element block's matrix is the Kronecker product
+ * of five 2x2 unit-determinant LU factors; the abstract: 15 parameters per
+ * block, fewer than half of per-channel scaling's 32).
  *   params [nb][15] fp32 -> T [nb][32][32] fp32, row-major:
  *   T[j][i][k] = prod_m A_jm[bit(i, 4-m)][bit(k, 4-m)]  (y_i = sum_k T[i][k] x_k).
  *   d = 32 * nb.  T 4-byte aligned.
@@ -241,7 +247,9 @@ int kq_gemm_mxfp4_rank1(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const
                         const float* mu, const float* wsum, float* Y, void* stream);
 
 /*
- * kq_dequant -- MXFP4 back to fp32, for checking:
+ * kq_dequant -- MXFP4 back to fp32, for checking (the abstract: W4A4 in
+ * MXFP4; the element value is the E2M1 code times the block's E8M0 scale,
+ * as the OCP Microscaling v1.0 format defines it):
  *   out[m][c] = E2M1(code) * 2^(scale - 127); scale 0xFF gives NaN.
  *   codes [M][d/2] (16-byte aligned), scales [M][d/32], out [M][d] fp32
  *   (16-byte aligned).  Values beyond the fp32 range (scale bytes 253, 254

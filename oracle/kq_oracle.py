@@ -304,6 +304,21 @@ def gemm_mxfp4(codes_a, scales_a, codes_b, scales_b) -> np.ndarray:
     return dequant(codes_a, scales_a) @ dequant(codes_b, scales_b).T
 
 
+def layer_error(x: np.ndarray, W: np.ndarray, params: np.ndarray) -> float:
+    """[ABS] the quantised W4A4 layer against the unquantised one, as one
+    number: ||Q(T x) Q(W T^-1)^T - x W^T||_F / ||x W^T||_F over the token rows
+    of x [M, d] and the weight rows of W [N, d], where Q is MXFP4 in
+    32-element blocks along d.  The pages learn the transform but state no
+    objective; this is the plain reading of "closer to the full-precision
+    output" (the quantity an offline fit of the parameters minimises)."""
+    x = np.asarray(x, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    ca, sa = kq_quantize(x, params)
+    cb, sb = quantize_weights(W, params)
+    ref = x @ W.T
+    return float(np.linalg.norm(gemm_mxfp4(ca, sa, cb, sb) - ref) / np.linalg.norm(ref))
+
+
 def gemm_error_scale(codes_a, scales_a, codes_b, scales_b) -> np.ndarray:
     """sum_k |a_k| |b_k| per output: the size of the terms an fp32
     accumulation adds up."""

@@ -451,6 +451,190 @@ def pin_undecided_flags(o):
 
 
 
+# --------------------------------------------------------------------------
+# the tolerance functions (they set every parity tolerance and exemption)
+# --------------------------------------------------------------------------
+def _mag_factor_by_hand(a, b, u):
+    """|L| |U| written out: |L| = [[1, 0], [|a|, 1]], |U| = [[|u|, |b|], [0, 1/|u|]],
+    so |L||U| = [[|u|, |b|], [|a||u|, |a||b| + 1/|u|]]."""
+    a, b, u = abs(float(a)), abs(float(b)), abs(float(u))
+    return [[u, b], [a * u, a * b + 1.0 / u]]
+
+
+def _inv_mag_factor_by_hand(a, b, u):
+    """|U^-1| |L^-1| written out: U^-1 = [[1/u, -b], [0, u]], L^-1 = [[1, 0], [-a, 1]],
+    so |U^-1||L^-1| = [[1/|u| + |b||a|, |b|], [|u||a|, |u|]]."""
+    a, b, u = abs(float(a)), abs(float(b)), abs(float(u))
+    return [[1.0 / u + b * a, b], [u * a, u]]
+
+
+def _kron_entry(F, i, k):
+    """Entry (i, k) of F[0] (x) ... (x) F[4] by the index-bit product."""
+    v = 1.0
+    for m in range(5):
+        s = 4 - m
+        v *= F[m][(i >> s) & 1][(k >> s) & 1]
+    return v
+
+
+def pin_error_scale_by_hand(o):
+    """One block worked by hand.  Factor 1 (the most significant index bit)
+    has a = 2, b = -3, u = 0.5; the others are the identity.  Then
+    |L||U| = [[0.5, 3], [1, 2*3 + 2]] = [[0.5, 3], [1, 8]] on bit 4, so for
+    x with x_0 = 1, x_16 = -2, x_5 = 4 and zeros elsewhere:
+      element 0:  0.5 |x_0| + 3 |x_16| = 0.5 + 6 = 6.5
+      element 16: 1 |x_0| + 8 |x_16| = 1 + 16 = 17
+      element 5:  0.5 |x_5| + 3 |x_21| = 2
+      element 21: 1 |x_5| + 8 |x_21| = 4
+    and 0 elsewhere.  Note |T| has 4 (= |2*(-3) + 2|) where |L||U| has 8: the
+    scale is the size of the summed terms, not of their (cancelling) sum."""
+    p = np.tile(np.array([0.0, 0.0, 1.0]), 5)
+    p[0:3] = [2.0, -3.0, 0.5]
+    x = np.zeros((1, 32))
+    x[0, 0], x[0, 16], x[0, 5] = 1.0, -2.0, 4.0
+    es = o.error_scale(x, p[None])
+    want = np.zeros((1, 32))
+    want[0, 0], want[0, 16], want[0, 5], want[0, 21] = 6.5, 17.0, 2.0, 4.0
+    assert np.array_equal(es, want), es
+    assert np.array_equal(o.lu_factor_magnitude(2.0, -3.0, 0.5), np.array([[0.5, 3.0], [1.0, 8.0]]))
+
+
+def pin_error_scale_definition(o):
+    """error_scale[m, 32 j + i] = sum_k ((x)_m |L_m||U_m|)[i, k] |x[m, 32 j + k]|,
+    rebuilt with plain loops (math.fsum) from the factor magnitudes written out
+    by hand; expand_magnitude against the same index-bit product."""
+    p = _rand_params(3, seed=71)
+    x = np.random.default_rng(72).normal(size=(4, 96)) * 3
+    es = o.error_scale(x, p)
+    em = o.expand_magnitude(p)
+    for j in range(3):
+        F = [_mag_factor_by_hand(*p[j, 3 * m:3 * m + 3]) for m in range(5)]
+        Tm = np.array([[_kron_entry(F, i, k) for k in range(32)] for i in range(32)])
+        assert np.allclose(em[j], Tm, rtol=1e-14, atol=0), j
+        for r in range(4):
+            for i in range(32):
+                ref = math.fsum(Tm[i, k] * abs(x[r, 32 * j + k]) for k in range(32))
+                assert abs(es[r, 32 * j + i] - ref) <= 1e-13 * ref, (r, j, i, es[r, 32 * j + i], ref)
+
+
+def pin_fold_error_scale(o):
+    """fold_error_scale[n, 32 j + i] = sum_k |W[n, 32 j + k]| ((x)_m |U_m^-1||L_m^-1|)[k, i]
+    (the folded weight is W T^-1, so the sum runs over the row index of T^-1),
+    by plain loops; and one entry by hand: factor 5 (least significant bit)
+    with a = 1, b = 2, u = 4, the rest identity, gives
+    |U^-1||L^-1| = [[1/4 + 2, 2], [4, 4]] on bit 0; for a row with w_0 = 1,
+    w_1 = -1: entry 0 = 1 * 2.25 + 1 * 4 = 6.25, entry 1 = 1 * 2 + 1 * 4 = 6."""
+    p = np.tile(np.array([0.0, 0.0, 1.0]), 5)
+    p[12:15] = [1.0, 2.0, 4.0]
+    W = np.zeros((1, 32))
+    W[0, 0], W[0, 1] = 1.0, -1.0
+    fe = o.fold_error_scale(W, p[None])
+    assert fe[0, 0] == 6.25 and fe[0, 1] == 6.0 and not fe[0, 2:].any(), fe
+    p = _rand_params(2, seed=73)
+    W = np.random.default_rng(74).normal(size=(3, 64))
+    fe = o.fold_error_scale(W, p)
+    for j in range(2):
+        F = [_inv_mag_factor_by_hand(*p[j, 3 * m:3 * m + 3]) for m in range(5)]
+        for n in range(3):
+            for i in range(32):
+                ref = math.fsum(abs(W[n, 32 * j + k]) * _kron_entry(F, k, i) for k in range(32))
+                assert abs(fe[n, 32 * j + i] - ref) <= 1e-13 * ref, (n, j, i)
+
+
+def pin_gemm_error_scale(o):
+    """gemm_error_scale[m, n] = sum_k |a_mk| |b_nk| over the decoded MXFP4
+    values, each decoded by hand from the E2M1 grid and 2^(byte - 127); and
+    one entry by hand: a row of codes 0x7 (6) and 0xF (-6) with scale 2^1
+    against codes 0x2 (1) with scale 2^-1 gives K * 12 * 0.5 = 6 K."""
+    rng = np.random.default_rng(75)
+    M, N, K = 3, 2, 96
+    ca = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    cb = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sa = rng.integers(120, 135, size=(M, K // 32), dtype=np.uint8)
+    sb = rng.integers(120, 135, size=(N, K // 32), dtype=np.uint8)
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+    def mag(codes, scales, r, k):
+        byte = int(codes[r, k // 2])
+        nib = (byte >> 4) if k % 2 else (byte & 15)
+        return grid[nib & 7] * 2.0 ** (int(scales[r, k // 32]) - 127)
+    G = o.gemm_error_scale(ca, sa, cb, sb)
+    for m in range(M):
+        for n in range(N):
+            assert G[m, n] == math.fsum(mag(ca, sa, m, k) * mag(cb, sb, n, k) for k in range(K))
+    ca1 = np.full((1, K // 2), 0xF7, dtype=np.uint8)
+    sa1 = np.full((1, K // 32), 128, dtype=np.uint8)
+    cb1 = np.full((1, K // 2), 0x22, dtype=np.uint8)
+    sb1 = np.full((1, K // 32), 126, dtype=np.uint8)
+    assert o.gemm_error_scale(ca1, sa1, cb1, sb1)[0, 0] == 6.0 * K
+
+
+def pin_undecided_tolerance_branches(o):
+    """The tolerance terms of the exemption rule, worked by hand.
+
+    Block A: amax = 22 (in [16, 32): floor(log2) = 4, e = 2, r = y / 4;
+      r = 5.5 and 0.65 for y = 22 and 2.6, far from every boundary).
+      y_1 = 4 * 1.251 = 5.004: r = 1.251 is 0.001 from the midpoint 1.25,
+      outside the relative window 1.25e-4.  The tolerance window is tol / 2^e:
+      tol = 0.003 gives 0.00075 (not flagged), tol = 0.005 gives 0.00125
+      (flagged).  (tol * 2^e or tol alone would flag both.)
+      y_2 = -0.001 lies 0.249 from the nearest midpoint in r; it is flagged
+      only through |y| <= tol: flagged for tol = 0.003, not for tol = 0.0005.
+    Block B: amax = 16.016, 0.016 above 2^4, outside the relative window
+      16e-4: the block is open for tol = 0.02, decided for tol = 0.01."""
+    y = np.zeros((1, 64))
+    y[0, 0] = 22.0
+    y[0, 1] = 4 * 1.251
+    y[0, 2] = -0.001
+    y[0, 3] = 2.6
+    y[0, 32] = 16.016
+    y[0, 33] = 1.3
+
+    def flags(tol_a, tol_b):
+        tol = np.zeros((1, 64))
+        tol[0, :32] = tol_a
+        tol[0, 32:] = tol_b
+        return o.undecided(y, tol)
+    e, b = flags(0.003, 0.01)
+    assert not e[0, 1] and e[0, 2] and not e[0, 0] and not e[0, 3]
+    assert not b[0, 0] and not b[0, 1] and not e[0, 33]
+    e, b = flags(0.005, 0.02)
+    assert e[0, 1] and b[0, 1] and e[0, 32:].all()
+    e, b = flags(0.0005, 0.0)
+    assert not e[0, 1] and not e[0, 2] and not b[0, 1]
+    # with a zero tolerance only the relative windows and exact zeros remain
+    e, b = o.undecided(y, np.zeros_like(y))
+    assert e[0, 4] and not e[0, 2] and not e[0, 1]
+
+
+def pin_layer_error_by_hand(o):
+    """The quantised layer's relative error, worked by hand on one 32-channel
+    block.  x = [7, 3, 0, ...], W = [[1, 0, ...], [0, 1, 0, ...]], identity
+    parameters: amax 7 gives e = 0, 7 saturates to 6 and 3 is on the grid, so
+    Q(x) = [6, 3, 0, ...]; W is exact.  x W^T = [7, 3], the quantised layer
+    gives [6, 3]: error 1 / sqrt(49 + 9) = 1 / sqrt(58).
+    With u = 2 on factor 1 (T = diag(2 x16, 1/2 x16)) the token becomes
+    [14, 6, ...]: e = 1, r = [7, 3] -> [6, 3], Q(T x) = [12, 6]; W T^-1 =
+    [[1/2, 0, ...], [0, 1/2, 0, ...]] is exact, so the layer gives [6, 3]
+    again: the same error.  u = 6/7 on factor 1 moves the outlier onto the
+    grid (T x = [6, 18/7]; amax 6, e = 0; 18/7 ~ 2.571 -> 3), but the folded
+    weights W T^-1 = [[7/6, 0, ...], [0, 7/6, 0, ...]] are quantised too:
+    amax 7/6 gives e = -2, r = 14/3 ~ 4.67 -> 4, i.e. 1.  The layer gives
+    [6 * 1, 3 * 1] = [6, 3] once more: error 1 / sqrt(58) (the weight side
+    takes back what the activation side gained)."""
+    x = np.zeros((1, 32))
+    x[0, 0], x[0, 1] = 7.0, 3.0
+    W = np.zeros((2, 32))
+    W[0, 0] = W[1, 1] = 1.0
+    ident = np.tile(np.array([0.0, 0.0, 1.0]), 5)[None]
+    assert abs(o.layer_error(x, W, ident) - 1.0 / math.sqrt(58.0)) < 1e-15
+    p = ident.copy()
+    p[0, 2] = 2.0
+    assert abs(o.layer_error(x, W, p) - 1.0 / math.sqrt(58.0)) < 1e-15
+    p[0, 2] = 6.0 / 7.0
+    assert abs(o.layer_error(x, W, p) - 1.0 / math.sqrt(58.0)) < 1e-15
+
+
 def pin_golden_hand_blocks(o):
     """The hand-worked blocks of tests/golden/kq_hand_blocks.txt: ties and
     saturation, the Kronecker factor order (a diagonal factor on the most and on

@@ -20,6 +20,15 @@ import oracle.kq_oracle as o
 TOL_REL = 1e-5        # transformed values: fp32 accumulation
 BOUNDARY_REL = 1e-4   # codes / scales: exemption window around a boundary
 
+# Exemption budget of a workload-sized comparison: the share of elements
+# whose decision the oracle leaves open, and the share left open only through
+# the evaluation tolerance (not by the 1e-4 window alone).  The synthetic
+# workloads sit near 0.07 % and 0.01 %; a tolerance that grew by an order of
+# magnitude, or a window computed on the wrong scale, would exceed these.
+EXEMPT_BUDGET = 3e-3
+TOL_ONLY_BUDGET = 5e-4
+BUDGET_MIN_ELEMS = 1 << 16    # smaller, hand-made cases are exempt from the budget
+
 
 @dataclasses.dataclass
 class Report:
@@ -30,11 +39,32 @@ class Report:
     code_mismatch: int = 0          # decided elements whose nibble differs
     exempt_blocks: int = 0
     exempt_elems: int = 0
+    exempt_tol_only: int = 0        # exempt only through the tolerance term
     differing_exempt: int = 0       # exempt elements that did differ (informational)
 
     @property
     def ok(self) -> bool:
         return self.y_violations == 0 and self.scale_mismatch == 0 and self.code_mismatch == 0
+
+    @property
+    def within_budget(self) -> bool:
+        """Exemptions bounded (only judged on workload-sized comparisons)."""
+        if self.n_elems < BUDGET_MIN_ELEMS:
+            return True
+        return (self.exempt_elems <= EXEMPT_BUDGET * self.n_elems
+                and self.exempt_tol_only <= TOL_ONLY_BUDGET * self.n_elems)
+
+    def counts(self) -> dict:
+        return {"elems": self.n_elems, "blocks": self.n_blocks,
+                "scale_mismatch": self.scale_mismatch, "code_mismatch": self.code_mismatch,
+                "y_violations": self.y_violations, "exempt_blocks": self.exempt_blocks,
+                "exempt_elems": self.exempt_elems, "exempt_tol_only": self.exempt_tol_only,
+                "differing_exempt": self.differing_exempt}
+
+    def assert_ok(self, label: str) -> None:
+        """Zero mismatches and exemptions within budget; the message carries
+        every count."""
+        assert self.ok and self.within_budget, f"{label}: {self.counts()}"
 
 
 def reference(x: np.ndarray, params=None, inv_s=None):
@@ -49,12 +79,13 @@ def reference(x: np.ndarray, params=None, inv_s=None):
     return y, tol
 
 
-def compare_codes(codes, scales, y_ref, tol, exact: bool = False) -> Report:
-    """Compare GPU (codes, scales) against the oracle's encoding of y_ref.
+def compare_codes(codes, scales, y_ref, tol, exact: bool = False, ref=None) -> Report:
+    """Compare GPU (codes, scales) against the oracle's encoding of y_ref
+    (or against ref = (codes, scales) the oracle produced from the same y_ref).
     exact=True: every decision must match (inputs whose transform is exact)."""
     codes = np.asarray(codes)
     scales = np.asarray(scales)
-    c_ref, s_ref = o.quantize_mxfp4(y_ref)
+    c_ref, s_ref = o.quantize_mxfp4(y_ref) if ref is None else ref
     M, d = y_ref.shape
     rep = Report(n_elems=M * d, n_blocks=M * d // 32)
     nan_blk = s_ref == o.E8M0_NAN
@@ -67,6 +98,8 @@ def compare_codes(codes, scales, y_ref, tol, exact: bool = False) -> Report:
     else:
         finite = np.where(np.isfinite(y_ref), y_ref, 0.0)
         e_flags, b_flags = o.undecided(finite, np.where(np.isfinite(tol), tol, 0.0))
+        e_rel, _ = o.undecided(finite, np.zeros_like(finite))
+        rep.exempt_tol_only = int(np.sum(e_flags & ~e_rel & np.repeat(~nan_blk, 32, axis=1)))
     rep.exempt_blocks = int(np.sum(b_flags & ~nan_blk))
     decided_blk = ~b_flags & ~nan_blk
     rep.scale_mismatch += int(np.sum(decided_blk & (scales != s_ref)))

@@ -141,3 +141,52 @@ def test_binding_refuses_host_tensors(lib):
         k.kq_quantize(x, p)
     with pytest.raises(ValueError, match="CUDA tensor"):
         k.kq_dequant(torch.zeros(4, 32, dtype=torch.uint8), torch.zeros(4, 2, dtype=torch.uint8))
+
+
+def test_binding_checks_array_sizes_and_devices(lib):
+    """The kernels read 15 parameters per 32-channel block (d inverse scales,
+    M offsets) through a raw pointer; an undersized array or one on another
+    device must be refused before anything is launched.  Sizes and devices
+    are checked before the CUDA check, so CPU tensors exercise them here."""
+    import torch
+    import w4a4_dit_post_b200 as k
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    good = torch.zeros(2, 15)
+    for bad in (torch.zeros(1, 15), torch.zeros(2, 14), torch.zeros(45)):
+        for fn in (k.kq_quantize, k.kq_quantize_sf_tiled, k.kq_transform):
+            with pytest.raises(ValueError, match="params has"):
+                fn(x, bad)
+        with pytest.raises(ValueError, match="params has"):
+            k.kq_quantize_tc(x, bad)
+        with pytest.raises(ValueError, match="params has"):
+            k.kq_quantize_centered(x, bad, torch.zeros(4))
+        with pytest.raises(ValueError, match="params has"):
+            k.kq_fold_weights(torch.zeros(3, 64), bad)
+        with pytest.raises(ValueError, match="params has"):
+            k.kq_quantize_weights(torch.zeros(3, 64), bad)
+    meta = torch.zeros(2, 15, device="meta")
+    with pytest.raises(ValueError, match="params is on meta"):
+        k.kq_quantize(x, meta)
+    with pytest.raises(ValueError, match="params is on meta"):
+        k.kq_quantize_weights(torch.zeros(3, 64), meta)
+    with pytest.raises(ValueError, match="inv_s has 63"):
+        k.sq_quantize(x, torch.zeros(63))
+    with pytest.raises(ValueError, match="inv_s is on meta"):
+        k.sq_quantize(x, torch.zeros(64, device="meta"))
+    with pytest.raises(ValueError, match="mu has 3"):
+        k.kq_quantize_centered(x, good, torch.zeros(3))
+    with pytest.raises(ValueError, match="mu is on meta"):
+        k.kq_quantize_centered(x, good, torch.zeros(4, device="meta"))
+    with pytest.raises(ValueError, match="positive multiple of 15"):
+        k.kq_expand_params(torch.zeros(16))
+    ca = torch.zeros(128, 64, dtype=torch.uint8)
+    ta = torch.zeros(1, 1, 512, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="wsum has 3"):
+        k.kq_gemm_mxfp4_rank1(ca, ta, ca, ta, torch.zeros(128), torch.zeros(3))
+    with pytest.raises(ValueError, match="b_codes is on meta"):
+        k.kq_gemm_mxfp4(ca, ta, ca.to("meta"), ta)
+    # well-formed CPU tensors get as far as the device check
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        k.kq_quantize(x, good)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        k.sq_quantize(x, torch.zeros(64))

@@ -48,3 +48,20 @@ def test_ncu_traffic_is_current_or_absent():
         # DRAM traffic of one launch: the input once plus part of the output, and
         # never more than the algorithmic bytes
         assert 4608 * 12288 * 2 <= traffic <= bench.algorithmic_bytes(4608, 12288)
+
+
+def test_both_arms_print_the_same_config():
+    cfg = bench.step_config(1)
+    assert cfg["M_per_rank"] == 4608 and cfg["d"] == [3072, 12288]
+    assert bench.step_config(1) == cfg
+
+
+def test_all_core_oracle_runner():
+    """Two spawned processes, two steps: every step's bytes are both
+    workers' tokens of both shapes plus the parameters."""
+    n, steps = bench.oracle_all_cores(rows_per_worker=4, steps=2, workers=2)
+    assert n == 2 and len(steps) == 2
+    want = 2 * 4 * (3072 + 12288) * bench.BYTES_PER_ELEM + (96 + 384) * bench.PARAM_BYTES_PER_BLOCK_COL
+    for secs, nbytes in steps:
+        assert secs > 0 and nbytes == want
+    assert bench.cpu_model() and bench.host_cores() >= 1

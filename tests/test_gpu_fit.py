@@ -59,3 +59,33 @@ def _smoothquant_error(kq, w, x_cal, x_test, W, ident):
     Y = kq.kq_gemm_mxfp4(c, kq.kq_sf_tile(sc), cw, kq.kq_sf_tile(sw))
     ref = x_test.float() @ W.t()
     return float(torch.linalg.norm(Y - ref) / torch.linalg.norm(ref))
+
+
+def test_layer_error_matches_oracle(kq):
+    """fit.layer_error (GPU quantizers, FP4 GEMM and torch's norm) against the
+    oracle's fp64 layer error on a 64 x 256 case.  Two checks: given the
+    GPU's own codes, the oracle's fp64 evaluation of the same error agrees
+    to fp32 accumulation accuracy; and against the oracle's end-to-end value
+    (its own quantisation) the difference stays within what the few exempt
+    rounding decisions can move it."""
+    import oracle.kq_oracle as o
+    from w4a4_dit_post_b200 import fit
+    w = synthetic.Workload("fit", 64, 256, "bf16", "normal", 0.02, None, 50.0, 2.0, 81)
+    raw = synthetic.make_activations(w)
+    x = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16).cuda()
+    X = synthetic.f32_from_bf16_bits(raw).astype(np.float64)
+    W = synthetic.make_weights(48, w.d, 82)
+    Wd = torch.from_numpy(W).cuda()
+    for p in (np.tile(fit.identity_block(), (w.nb, 1)), np.tile(fit.hadamard_block(), (w.nb, 1)),
+              synthetic.make_params(w.nb, 83)):
+        pd = torch.from_numpy(np.ascontiguousarray(p, dtype=np.float32)).cuda()
+        e_gpu = fit.layer_error(x, Wd, pd)
+        ca, sa = kq.kq_quantize(x, pd)
+        cb, sb = kq.kq_quantize_weights(Wd, pd)
+        ca, sa, cb, sb = (t.cpu().numpy() for t in (ca, sa, cb, sb))
+        ref = X @ W.astype(np.float64).T
+        e_same_codes = np.linalg.norm(o.gemm_mxfp4(ca, sa, cb, sb) - ref) / np.linalg.norm(ref)
+        e_oracle = o.layer_error(X, W, p)
+        print(f"layer error: gpu {e_gpu:.6f}, oracle on gpu codes {e_same_codes:.6f}, oracle {e_oracle:.6f}")
+        assert abs(e_gpu - e_same_codes) <= 1e-4 * e_same_codes
+        assert abs(e_gpu - e_oracle) <= 2e-3 * e_oracle

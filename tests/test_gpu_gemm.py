@@ -154,3 +154,56 @@ def test_quantize_with_tiled_scales(kq, M, d):
     kq.kq_quantize_sf_tiled(x, p, c2, t2)
     torch.cuda.synchronize()
     assert torch.equal(c1, c2) and torch.equal(t1, t2)
+
+
+# ---------------------------------------------------------------------------
+# the persistent schedule: more 128 x 128 output tiles than CTAs (two per SM
+# on 148 SMs = 296), so every CTA walks two or more tiles and the stage ring
+# and the accumulator hand-back carry over from one tile to the next
+# ---------------------------------------------------------------------------
+MULTI_TILE = [(2048, 2560, 1024), (2176, 2304, 512), (4608, 3072, 3072)]   # 320, 306, 864 tiles
+
+
+def _sampled_rows(M, n, seed):
+    if M <= n:
+        return np.arange(M)
+    rng = np.random.default_rng([seed, M])
+    return np.unique(np.concatenate([[0, M - 1], rng.choice(M, n, replace=False)]))
+
+
+@pytest.mark.parametrize("M,N,K", MULTI_TILE)
+def test_gemm_persistent_unit_scales_exact(kq, M, N, K):
+    """Unit scales keep every sum exact in fp32 (|sum| <= 36 K, a multiple of
+    1/4: at most 19 significant bits here), so each sampled row must equal
+    the oracle bit for bit, whichever CTA and tile produced it."""
+    rng = np.random.default_rng(M + N + K)
+    ca, sa = _operands(rng, M, K, 127, 127)
+    cb, sb = _operands(rng, N, K, 127, 127)
+    Y = _gemm(kq, ca, sa, cb, sb)
+    rows = _sampled_rows(M, 256, K)
+    assert np.array_equal(Y[rows], o.gemm_mxfp4(ca[rows], sa[rows], cb, sb))
+
+
+@pytest.mark.parametrize("M,N,K", MULTI_TILE)
+def test_gemm_persistent_scaled_matches_oracle(kq, M, N, K):
+    """Scales 2^-10 .. 2^10, fp32 and bf16 outputs and the rank-1 epilogue,
+    on sampled rows x all columns (every tile column), within the fp32
+    accumulation bound of the fp64 oracle."""
+    rng = np.random.default_rng(3 * M + N + K)
+    ca, sa = _operands(rng, M, K, 117, 137)
+    cb, sb = _operands(rng, N, K, 117, 137)
+    ta, tb = kq.kq_sf_tile(_cuda(sa)), kq.kq_sf_tile(_cuda(sb))
+    da, db = _cuda(ca), _cuda(cb)
+    mu = rng.normal(0, 4, size=M).astype(np.float32)
+    wsum = rng.normal(0, 1, size=N).astype(np.float32)
+    Y = kq.kq_gemm_mxfp4(da, ta, db, tb).cpu().numpy().astype(np.float64)
+    Y16 = kq.kq_gemm_mxfp4_bf16(da, ta, db, tb).cpu().to(torch.float64).numpy()
+    Y1 = kq.kq_gemm_mxfp4_rank1(da, ta, db, tb, _cuda(mu), _cuda(wsum)).cpu().numpy().astype(np.float64)
+    rows = _sampled_rows(M, 256, K + 1)
+    ref = o.gemm_mxfp4(ca[rows], sa[rows], cb, sb)
+    tol = (K / 64 + 64) * 2.0 ** -23 * o.gemm_error_scale(ca[rows], sa[rows], cb, sb)
+    assert np.all(np.abs(Y[rows] - ref) <= tol)
+    assert np.all(np.abs(Y16[rows] - ref) <= tol + 2.0 ** -8 * (np.abs(ref) + tol))
+    ref1 = o.gemm_mxfp4_rank1(ca[rows], sa[rows], cb, sb, mu[rows], wsum)
+    tol1 = tol + 2.0 ** -22 * (np.abs(np.outer(mu[rows], wsum)) + np.abs(ref1))
+    assert np.all(np.abs(Y1[rows] - ref1) <= tol1)

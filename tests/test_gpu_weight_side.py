@@ -31,10 +31,8 @@ def kq():
 
 
 def check(rep, label):
-    print(f"{label}: blocks={rep.n_blocks} scale_mismatch={rep.scale_mismatch} "
-          f"code_mismatch={rep.code_mismatch} exempt_blocks={rep.exempt_blocks} "
-          f"exempt_elems={rep.exempt_elems} differing_exempt={rep.differing_exempt}")
-    assert rep.ok, label
+    print(f"{label}: {rep.counts()}")
+    rep.assert_ok(label)
 
 
 # (N, d): tiny and ragged shapes, then the FLUX.1-schnell layer shapes

@@ -152,6 +152,74 @@ def m_centering_after_transform(o):
         o.transform(np.asarray(x, dtype=np.float64), params) - np.asarray(mu, dtype=np.float64)[:, None])
 
 
+# the tolerance functions: each scaled by 10, or a term dropped or misplaced
+def m_error_scale_x10(o):
+    f = o.error_scale
+    o.error_scale = lambda x, params: 10.0 * f(x, params)
+
+
+def m_expand_magnitude_x10(o):
+    f = o.expand_magnitude
+    o.expand_magnitude = lambda params: 10.0 * f(params)
+
+
+def m_lu_factor_magnitude_x10(o):
+    f = o.lu_factor_magnitude
+    o.lu_factor_magnitude = lambda a, b, u: 10.0 * f(a, b, u)
+
+
+def m_error_scale_uses_abs_T(o):
+    o.expand_magnitude = lambda params: np.abs(o.expand_params(params))
+
+
+def m_fold_error_scale_x10(o):
+    f = o.fold_error_scale
+    o.fold_error_scale = lambda W, params: 10.0 * f(W, params)
+
+
+def m_gemm_error_scale_x10(o):
+    f = o.gemm_error_scale
+    o.gemm_error_scale = lambda *a: 10.0 * f(*a)
+
+
+def m_undecided_tol_x10(o):
+    f = o.undecided
+    o.undecided = lambda y, tol, rel=1e-4: f(y, 10.0 * np.asarray(tol), rel)
+
+
+def m_undecided_rel_x10(o):
+    f = o.undecided
+    o.undecided = lambda y, tol, rel=1e-4: f(y, tol, 10.0 * rel)
+
+
+def m_undecided_tol_times_scale(o):
+    """tol * 2^e instead of tol / 2^e in the element window."""
+    src = open(ORACLE_PATH).read()
+    assert "tr = np.ldexp(tb, -e[:, :, None])" in src
+    ns = {}
+    exec(compile(src.replace("tr = np.ldexp(tb, -e[:, :, None])", "tr = np.ldexp(tb, e[:, :, None])"),
+                 ORACLE_PATH, "exec"), ns)
+    o.undecided = ns["undecided"]
+
+
+def m_undecided_no_sign_branch(o):
+    src = open(ORACLE_PATH).read()
+    assert "elem |= np.abs(yb) <= tb" in src
+    ns = {}
+    exec(compile(src.replace("elem |= np.abs(yb) <= tb", "pass"), ORACLE_PATH, "exec"), ns)
+    o.undecided = ns["undecided"]
+
+
+
+def m_layer_error_unfolded_weights(o):
+    def le(x, W, params):
+        ca, sa = o.kq_quantize(np.asarray(x, dtype=np.float64), params)
+        cb, sb = o.quantize_mxfp4(np.asarray(W, dtype=np.float64))
+        ref = np.asarray(x, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T
+        return float(np.linalg.norm(o.gemm_mxfp4(ca, sa, cb, sb) - ref) / np.linalg.norm(ref))
+    o.layer_error = le
+
+
 MUTANTS = [v for k, v in sorted(globals().items()) if k.startswith("m_")]
 
 

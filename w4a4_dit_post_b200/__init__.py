@@ -1,9 +1,13 @@
 """Python binding of the KroQuant C ABI (``include/kq.h``, ``libkroquant.so``).
 
 Argument marshalling only: every function checks that it was handed CUDA
-tensors of the right dtype and shape, allocates missing outputs with torch
-(device memory is PyTorch's job here), and passes raw device pointers and the
-current torch stream to the C function of the same name.  All arithmetic runs
+tensors of the right dtype and shape, that every array the kernels read
+through a raw pointer (parameters, inverse scales, offsets, row sums) holds
+exactly the number of elements the call reads and sits on the same device as
+the activations, allocates missing outputs with torch (device memory is
+PyTorch's job here), and passes raw device pointers and the current torch
+stream to the C function of the same name.  Sizes and devices are checked
+before the CUDA check, so the checks also run on tensors of any device.  All arithmetic runs
 in the library's sm_100a kernels; there is no CPU path.  If the library has
 not been built, the first call raises ``RuntimeError`` (build it with
 ``python -m w4a4_dit_post_b200.build``).
@@ -111,17 +115,40 @@ def _stream(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
-def _need_cuda(name: str, t: torch.Tensor, dtypes, ndim: int | None = None) -> None:
+def _need(name: str, t: torch.Tensor, dtypes, ndim: int | None = None) -> None:
+    """Type, dtype, rank and contiguity of a tensor argument (any device)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor (the library takes device pointers)")
     if t.dtype not in dtypes:
         raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _need_cuda(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library takes device pointers)")
+
+
+def _same_device(name: str, t: torch.Tensor, like: torch.Tensor, like_name: str) -> None:
+    if t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, {like_name} on {like.device}")
+
+
+def _need_numel(name: str, t: torch.Tensor, n: int, what: str) -> None:
+    # the kernels read exactly n elements through the raw pointer: a shorter
+    # tensor would be read out of bounds
+    if t.numel() != n:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {n} ({what})")
+
+
+def _need_params(params: torch.Tensor, d: int, like: torch.Tensor, like_name: str = "x") -> None:
+    """LU parameters: fp32, exactly 15 per 32-channel block of d, on like's device."""
+    _need("params", params, (torch.float32,))
+    _need_numel("params", params, 15 * (d // 32), f"15 LU parameters per 32-channel block of d = {d}")
+    _same_device("params", params, like, like_name)
 
 
 def _x_dtype(x: torch.Tensor) -> int:
@@ -131,23 +158,29 @@ def _x_dtype(x: torch.Tensor) -> int:
 def _out(t, shape, dtype, like, name):
     if t is None:
         return torch.empty(shape, dtype=dtype, device=like.device)
-    _need_cuda(name, t, (dtype,))
+    _need(name, t, (dtype,))
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
-    if t.device != like.device:
-        raise ValueError(f"{name} is on {t.device}, inputs on {like.device}")
+    _same_device(name, t, like, "the inputs")
     return t
 
 
 _ACT = (torch.bfloat16, torch.float32)
 
 
+def _activation(x, dtypes=_ACT):
+    """x [M, d]: dtype, rank, contiguity; returns (M, d).  d is checked by
+    the library (a positive multiple of 32)."""
+    _need("x", x, dtypes, 2)
+    return x.shape
+
+
 def kq_quantize(x, params, codes=None, scales=None):
     """KroQuant quantizer: x [M, d] bf16/fp32, params [d/32, 15] fp32 ->
     (codes uint8 [M, d/2], scales uint8 [M, d/32])."""
-    _need_cuda("x", x, _ACT, 2)
-    _need_cuda("params", params, (torch.float32,))
-    M, d = x.shape
+    M, d = _activation(x)
+    _need_params(params, d, x)
+    _need_cuda("x", x)
     codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
     scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
     with torch.cuda.device(x.device):
@@ -160,9 +193,9 @@ def kq_quantize(x, params, codes=None, scales=None):
 def kq_quantize_sf_tiled(x, params, codes=None, scales_tiled=None):
     """kq_quantize with the scales in the blocked layout kq_gemm_mxfp4 reads:
     (codes uint8 [M, d/2], scales_tiled uint8 [ceil(M/128), d/128, 512])."""
-    _need_cuda("x", x, _ACT, 2)
-    _need_cuda("params", params, (torch.float32,))
-    M, d = x.shape
+    M, d = _activation(x)
+    _need_params(params, d, x)
+    _need_cuda("x", x)
     codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
     scales_tiled = _out(scales_tiled, ((M + 127) // 128, d // 128 if d % 128 == 0 else 0, 512),
                         torch.uint8, x, "scales_tiled")
@@ -176,9 +209,9 @@ def kq_quantize_sf_tiled(x, params, codes=None, scales_tiled=None):
 def kq_quantize_tc(x, params, codes=None, scales=None):
     """Same result contract as kq_quantize, computed on the tensor cores
     (bf16 input only); kept for comparison with the SIMT path."""
-    _need_cuda("x", x, (torch.bfloat16,), 2)
-    _need_cuda("params", params, (torch.float32,))
-    M, d = x.shape
+    M, d = _activation(x, (torch.bfloat16,))
+    _need_params(params, d, x)
+    _need_cuda("x", x)
     codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
     scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
     with torch.cuda.device(x.device):
@@ -190,9 +223,9 @@ def kq_quantize_tc(x, params, codes=None, scales=None):
 
 def kq_transform(x, params, y=None):
     """Transform stage alone: y = blockdiag(T_j) x, fp32 [M, d]."""
-    _need_cuda("x", x, _ACT, 2)
-    _need_cuda("params", params, (torch.float32,))
-    M, d = x.shape
+    M, d = _activation(x)
+    _need_params(params, d, x)
+    _need_cuda("x", x)
     y = _out(y, (M, d), torch.float32, x, "y")
     with torch.cuda.device(x.device):
         _check("kq_transform", abi().kq_transform(
@@ -202,9 +235,11 @@ def kq_transform(x, params, y=None):
 
 def sq_quantize(x, inv_s, codes=None, scales=None):
     """SmoothQuant comparison quantizer: y_c = x_c * inv_s[c], then MXFP4."""
-    _need_cuda("x", x, _ACT, 2)
-    _need_cuda("inv_s", inv_s, (torch.float32,), 1)
-    M, d = x.shape
+    M, d = _activation(x)
+    _need("inv_s", inv_s, (torch.float32,), 1)
+    _need_numel("inv_s", inv_s, d, "one inverse scale per channel")
+    _same_device("inv_s", inv_s, x, "x")
+    _need_cuda("x", x)
     codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
     scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
     with torch.cuda.device(x.device):
@@ -216,7 +251,10 @@ def sq_quantize(x, inv_s, codes=None, scales=None):
 
 def kq_expand_params(params, T=None):
     """params [nb, 15] -> T [nb, 32, 32] fp32."""
-    _need_cuda("params", params, (torch.float32,))
+    _need("params", params, (torch.float32,))
+    if params.numel() == 0 or params.numel() % 15:
+        raise ValueError(f"params has {params.numel()} elements, expected a positive multiple of 15")
+    _need_cuda("params", params)
     nb = params.numel() // 15
     T = _out(T, (nb, 32, 32), torch.float32, params, "T")
     with torch.cuda.device(params.device):
@@ -227,9 +265,10 @@ def kq_expand_params(params, T=None):
 
 def kq_fold_weights(W, params, W_out=None):
     """W [N, d] fp32 -> W blockdiag(T_j)^{-1}.  Pass W_out=W for in place."""
-    _need_cuda("W", W, (torch.float32,), 2)
-    _need_cuda("params", params, (torch.float32,))
+    _need("W", W, (torch.float32,), 2)
     N, d = W.shape
+    _need_params(params, d, W, "W")
+    _need_cuda("W", W)
     W_out = _out(W_out, (N, d), torch.float32, W, "W_out")
     with torch.cuda.device(W.device):
         _check("kq_fold_weights", abi().kq_fold_weights(
@@ -240,9 +279,10 @@ def kq_fold_weights(W, params, W_out=None):
 def kq_quantize_weights(W, params, codes=None, scales=None):
     """Weight side: W [N, d] fp32 -> MXFP4 (codes uint8 [N, d/2], scales
     uint8 [N, d/32]) of the folded weights W blockdiag(T_j)^{-1}."""
-    _need_cuda("W", W, (torch.float32,), 2)
-    _need_cuda("params", params, (torch.float32,))
+    _need("W", W, (torch.float32,), 2)
     N, d = W.shape
+    _need_params(params, d, W, "W")
+    _need_cuda("W", W)
     codes = _out(codes, (N, d // 2), torch.uint8, W, "codes")
     scales = _out(scales, (N, d // 32), torch.uint8, W, "scales")
     with torch.cuda.device(W.device):
@@ -254,7 +294,8 @@ def kq_quantize_weights(W, params, codes=None, scales=None):
 def kq_sf_tile(scales, out=None):
     """Scale bytes [R, K/32] -> the blocked layout [ceil(R/128), K/128, 512]
     that kq_gemm_mxfp4 reads."""
-    _need_cuda("scales", scales, (torch.uint8,), 2)
+    _need("scales", scales, (torch.uint8,), 2)
+    _need_cuda("scales", scales)
     R, ns = scales.shape
     K = 32 * ns
     out = _out(out, ((R + 127) // 128, K // 128 if K % 128 == 0 else 0, 512), torch.uint8, scales, "out")
@@ -265,9 +306,9 @@ def kq_sf_tile(scales, out=None):
 
 def _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled):
     for name, t in (("a_codes", a_codes), ("b_codes", b_codes)):
-        _need_cuda(name, t, (torch.uint8,), 2)
+        _need(name, t, (torch.uint8,), 2)
     for name, t in (("a_sf_tiled", a_sf_tiled), ("b_sf_tiled", b_sf_tiled)):
-        _need_cuda(name, t, (torch.uint8,), 3)
+        _need(name, t, (torch.uint8,), 3)
     M, half = a_codes.shape
     N = b_codes.shape[0]
     K = 2 * half
@@ -277,6 +318,8 @@ def _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled):
         if tuple(t.shape) != ((rows + 127) // 128, K // 128, 512):
             raise ValueError(f"{name} has shape {tuple(t.shape)}, expected "
                              f"{((rows + 127) // 128, K // 128, 512)}")
+    for name, t in (("a_sf_tiled", a_sf_tiled), ("b_codes", b_codes), ("b_sf_tiled", b_sf_tiled)):
+        _same_device(name, t, a_codes, "a_codes")
     return M, N, K
 
 
@@ -284,6 +327,7 @@ def kq_gemm_mxfp4(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
     """Y [M, N] fp32 = MXFP4(A) MXFP4(B)^T from codes [M, K/2] / [N, K/2] and
     scales tiled by kq_sf_tile."""
     M, N, K = _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled)
+    _need_cuda("a_codes", a_codes)
     Y = _out(Y, (M, N), torch.float32, a_codes, "Y")
     with torch.cuda.device(a_codes.device):
         _check("kq_gemm_mxfp4", abi().kq_gemm_mxfp4(
@@ -295,6 +339,7 @@ def kq_gemm_mxfp4(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
 def kq_gemm_mxfp4_bf16(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
     """kq_gemm_mxfp4 with Y [M, N] bf16 (each fp32 sum rounded to nearest even)."""
     M, N, K = _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled)
+    _need_cuda("a_codes", a_codes)
     Y = _out(Y, (M, N), torch.bfloat16, a_codes, "Y")
     with torch.cuda.device(a_codes.device):
         _check("kq_gemm_mxfp4_bf16", abi().kq_gemm_mxfp4_bf16(
@@ -305,8 +350,8 @@ def kq_gemm_mxfp4_bf16(a_codes, a_sf_tiled, b_codes, b_sf_tiled, Y=None):
 
 def kq_row_sum(x, scale=1.0, out=None):
     """out [M] fp32 = scale * row sums of x [M, d] (bf16 or fp32)."""
-    _need_cuda("x", x, _ACT, 2)
-    M, d = x.shape
+    M, d = _activation(x)
+    _need_cuda("x", x)
     out = _out(out, (M,), torch.float32, x, "out")
     with torch.cuda.device(x.device):
         _check("kq_row_sum", abi().kq_row_sum(x.data_ptr(), _x_dtype(x), M, d, float(scale),
@@ -316,12 +361,12 @@ def kq_row_sum(x, scale=1.0, out=None):
 
 def kq_quantize_centered(x, params, mu, codes=None, scales=None):
     """Centring variant: MXFP4(T (x - mu 1)) with mu [M] fp32 per-token offsets."""
-    _need_cuda("x", x, _ACT, 2)
-    _need_cuda("params", params, (torch.float32,))
-    _need_cuda("mu", mu, (torch.float32,), 1)
-    M, d = x.shape
-    if mu.shape[0] != M:
-        raise ValueError("mu must have one offset per row of x")
+    M, d = _activation(x)
+    _need_params(params, d, x)
+    _need("mu", mu, (torch.float32,), 1)
+    _need_numel("mu", mu, M, "one offset per row of x")
+    _same_device("mu", mu, x, "x")
+    _need_cuda("x", x)
     codes = _out(codes, (M, d // 2), torch.uint8, x, "codes")
     scales = _out(scales, (M, d // 32), torch.uint8, x, "scales")
     with torch.cuda.device(x.device):
@@ -333,17 +378,14 @@ def kq_quantize_centered(x, params, mu, codes=None, scales=None):
 
 def kq_gemm_mxfp4_rank1(a_codes, a_sf_tiled, b_codes, b_sf_tiled, mu, wsum, Y=None):
     """kq_gemm_mxfp4 plus mu wsum^T (mu [M], wsum [N] fp32)."""
-    for name, t in (("a_codes", a_codes), ("b_codes", b_codes)):
-        _need_cuda(name, t, (torch.uint8,), 2)
-    for name, t in (("a_sf_tiled", a_sf_tiled), ("b_sf_tiled", b_sf_tiled)):
-        _need_cuda(name, t, (torch.uint8,), 3)
-    _need_cuda("mu", mu, (torch.float32,), 1)
-    _need_cuda("wsum", wsum, (torch.float32,), 1)
-    M, half = a_codes.shape
-    N = b_codes.shape[0]
-    K = 2 * half
-    if b_codes.shape[1] != half or mu.shape[0] != M or wsum.shape[0] != N:
-        raise ValueError("operand shapes disagree")
+    M, N, K = _gemm_shapes(a_codes, a_sf_tiled, b_codes, b_sf_tiled)
+    _need("mu", mu, (torch.float32,), 1)
+    _need("wsum", wsum, (torch.float32,), 1)
+    _need_numel("mu", mu, M, "one offset per activation row")
+    _need_numel("wsum", wsum, N, "one row sum per weight row")
+    _same_device("mu", mu, a_codes, "a_codes")
+    _same_device("wsum", wsum, a_codes, "a_codes")
+    _need_cuda("a_codes", a_codes)
     Y = _out(Y, (M, N), torch.float32, a_codes, "Y")
     with torch.cuda.device(a_codes.device):
         _check("kq_gemm_mxfp4_rank1", abi().kq_gemm_mxfp4_rank1(
@@ -354,12 +396,14 @@ def kq_gemm_mxfp4_rank1(a_codes, a_sf_tiled, b_codes, b_sf_tiled, mu, wsum, Y=No
 
 def kq_dequant(codes, scales, out=None):
     """MXFP4 -> fp32 [M, d]."""
-    _need_cuda("codes", codes, (torch.uint8,), 2)
-    _need_cuda("scales", scales, (torch.uint8,), 2)
+    _need("codes", codes, (torch.uint8,), 2)
+    _need("scales", scales, (torch.uint8,), 2)
     M, half = codes.shape
     d = 2 * half
     if tuple(scales.shape) != (M, d // 32):
         raise ValueError("scales shape does not match codes")
+    _same_device("scales", scales, codes, "codes")
+    _need_cuda("codes", codes)
     out = _out(out, (M, d), torch.float32, codes, "out")
     with torch.cuda.device(codes.device):
         _check("kq_dequant", abi().kq_dequant(
