@@ -87,7 +87,7 @@ extern "C" {
  *   scales  [M][d/32] uint8 output; any alignment.
  * For each token row and block j: y = T_j x_j in fp32 arithmetic, then MXFP4
  * (the abstract: transform the activations, then quantise; W4A4 in MXFP4).
- * Limits: d <= KQ_MAX_D; M * d / 32 < 2^31.
+ * Limits: d <= KQ_MAX_D; M * d / 32 < 2^31; M < 2^30 (KQ_ERR_UNSUPPORTED).
  */
 int kq_quantize(const void* x, int x_dtype, int64_t M, int64_t d,
                 const float* params, uint8_t* codes, uint8_t* scales,

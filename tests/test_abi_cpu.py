@@ -80,6 +80,8 @@ def test_quantize_argument_checks(lib):
     assert q(A16, 0, 4, 64, A16b, A16c + 4, A16d, None) == 2       # codes alignment
     assert q(A16, 0, 4, 32768 + 32, A16b, A16c, A16d, None) == 4   # d limit
     assert q(A16, 0, 2 ** 40, 1024, A16b, A16c, A16d, None) == 4   # block count
+    assert q(A16, 0, 2 ** 30, 32, A16b, A16c, A16d, None) == 4     # row count (M < 2^30)
+    assert lib.sq_quantize(A16, 0, 2 ** 30, 32, A16b, A16c, A16d, None) == 4
     assert q(A16, 0, 0, 64, A16b, A16c, A16d + 1, None) == 0       # M == 0: no-op
     assert q(None, 0, 0, 64, None, None, None, None) == 0          # ... pointers unused
     assert q(None, 0, 0, 48, None, None, None, None) == 1          # shape still checked

@@ -377,9 +377,12 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   // kStages tiles (a counter and a flag instead of a division per tile).
   int rt = rt_first;
   uint32_t parity = 0;
-  // this thread's row, and its output block, advanced by a constant per tile
-  int r0 = rt_first * R + rr;
-  const int r_step = row_step * R;
+  // This thread's row (unsigned: the host refuses M >= 2^30, so it stays
+  // below 2^31 + 2^9 even one step past the last tile) and its output block,
+  // advanced by a constant per tile; the output pointers move only while
+  // another tile follows, so they never point past their buffers.
+  uint32_t r0 = (uint32_t)(rt_first * R + rr);
+  const uint32_t r_step = (uint32_t)(row_step * R);
   const size_t g_first = (size_t)r0 * nb + j0 + c, g_step = (size_t)r_step * nb;
   constexpr bool kCodes = kOp != Op::kKqTransform;   // the other output is NULL
   uint8_t* cdst = kCodes ? codes + g_first * 16 : nullptr;
@@ -387,13 +390,13 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   float* ydst = kCodes ? nullptr : y_out + g_first * 32;
   for (;;) {
 #pragma unroll 1
-    for (int s = 0; s < kStages; ++s, rt += row_step, r0 += r_step) {
+    for (int s = 0; s < kStages; ++s) {
       if (rt >= geo.n_row_tiles) return;
       float2 v[16];
       // centring variant: this row's offset (read before the wait, so the
       // load overlaps it)
       float2 neg_mu = make_float2(0.0f, 0.0f);
-      if (kOp == Op::kKqCentered && active && r0 < geo.M) neg_mu = make_float2(-mu[r0], -mu[r0]);
+      if (kOp == Op::kKqCentered && active && r0 < (uint32_t)geo.M) neg_mu = make_float2(-mu[r0], -mu[r0]);
       const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity);
       if (ok) {
         if (active) {
@@ -427,13 +430,17 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
           tma_load_3d(smem_addr(smem + s * stage_bytes), &tmap, 0, j0, nrt * R, smem_addr(&bars[s]));
         }
       }
-      if (active && r0 < geo.M)
-        quantize_row<kOp>(v, crow, geo, r0, j0 + c, cdst, sdst, ydst, scales);
-      if constexpr (kCodes) {
-        cdst += g_step * 16;
-        sdst += g_step;
-      } else {
-        ydst += g_step * 32;
+      if (active && r0 < (uint32_t)geo.M)
+        quantize_row<kOp>(v, crow, geo, (int)r0, j0 + c, cdst, sdst, ydst, scales);
+      rt += row_step;
+      r0 += r_step;
+      if (rt < geo.n_row_tiles) {
+        if constexpr (kCodes) {
+          cdst += g_step * 16;
+          sdst += g_step;
+        } else {
+          ydst += g_step * 32;
+        }
       }
     }
     parity ^= 1u;
@@ -565,6 +572,8 @@ int dispatch(const void* x, int x_dtype, int64_t M, int64_t d, const float* coef
              uint8_t* codes, uint8_t* scales, float* y, void* stream, const char* fn,
              bool sf_tiled = false, const float* mu = nullptr, bool need_mu = false) {
   if (int st = check_shape(M, d, KQ_MAX_D, fn)) return st;
+  if (M >= ((int64_t)1 << 30))
+    return fail(KQ_ERR_UNSUPPORTED, "%s: M = %lld rows exceeds the limit 2^30 - 1", fn, (long long)M);
   if (sf_tiled && d % 128 != 0)
     return fail(KQ_ERR_INVALID_ARG, "%s: d must be a multiple of 128 (d = %lld)", fn, (long long)d);
   if (x_dtype != KQ_DTYPE_BF16 && x_dtype != KQ_DTYPE_F32)
