@@ -378,19 +378,21 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
   int rt = rt_first;
   uint32_t parity = 0;
   // This thread's row (unsigned: the host refuses M >= 2^30, so it stays
-  // below 2^31 + 2^9 even one step past the last tile) and its output block,
-  // advanced by a constant per tile; the output pointers move only while
-  // another tile follows, so they never point past their buffers.
+  // below 2^31 + 2^9 even one step past the last tile) and the addresses of
+  // its output block, advanced by a constant per tile.  The addresses are
+  // kept as integers: after the last tile they step past the buffers, and
+  // unsigned arithmetic makes that well defined; they are only dereferenced
+  // for rows below M.
   uint32_t r0 = (uint32_t)(rt_first * R + rr);
   const uint32_t r_step = (uint32_t)(row_step * R);
   const size_t g_first = (size_t)r0 * nb + j0 + c, g_step = (size_t)r_step * nb;
   constexpr bool kCodes = kOp != Op::kKqTransform;   // the other output is NULL
-  uint8_t* cdst = kCodes ? codes + g_first * 16 : nullptr;
-  uint8_t* sdst = kCodes ? scales + g_first : nullptr;
-  float* ydst = kCodes ? nullptr : y_out + g_first * 32;
+  uintptr_t cdst = kCodes ? reinterpret_cast<uintptr_t>(codes) + g_first * 16 : 0;
+  uintptr_t sdst = kCodes ? reinterpret_cast<uintptr_t>(scales) + g_first : 0;
+  uintptr_t ydst = kCodes ? 0 : reinterpret_cast<uintptr_t>(y_out) + g_first * 128;
   for (;;) {
 #pragma unroll 1
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStages; ++s, rt += row_step, r0 += r_step) {
       if (rt >= geo.n_row_tiles) return;
       float2 v[16];
       // centring variant: this row's offset (read before the wait, so the
@@ -431,16 +433,13 @@ stream_kernel(const __grid_constant__ CUtensorMap tmap, const float* __restrict_
         }
       }
       if (active && r0 < (uint32_t)geo.M)
-        quantize_row<kOp>(v, crow, geo, (int)r0, j0 + c, cdst, sdst, ydst, scales);
-      rt += row_step;
-      r0 += r_step;
-      if (rt < geo.n_row_tiles) {
-        if constexpr (kCodes) {
-          cdst += g_step * 16;
-          sdst += g_step;
-        } else {
-          ydst += g_step * 32;
-        }
+        quantize_row<kOp>(v, crow, geo, (int)r0, j0 + c, reinterpret_cast<uint8_t*>(cdst),
+                          reinterpret_cast<uint8_t*>(sdst), reinterpret_cast<float*>(ydst), scales);
+      if constexpr (kCodes) {
+        cdst += g_step * 16;
+        sdst += g_step;
+      } else {
+        ydst += g_step * 128;
       }
     }
     parity ^= 1u;
