@@ -463,7 +463,8 @@ def time_gemm(kq, device, stream, K_launches: int, W: int, shapes=None) -> dict:
     import torch
     lib = kq.abi()
     peak, src = fp4_peak()
-    out = {"kernel": "kq_gemm_mxfp4 (tcgen05 kind::mxf4 block32; fp32 out, and bf16 out: kq_gemm_mxfp4_bf16)",
+    out = {"kernel": "kq_gemm_mxfp4 (tcgen05 kind::mxf4 block32, 256 x 256 tiles over SM pairs; fp32 out, "
+                     "and bf16 out: kq_gemm_mxfp4_bf16); cuBLAS block-scaled FP4 (scaled_mm) timed beside it",
            "peak_tflops": round(peak, 1),
            "peak_source": src, "shapes": {}}
     g = torch.Generator(device=device)
@@ -496,6 +497,33 @@ def time_gemm(kq, device, stream, K_launches: int, W: int, shapes=None) -> dict:
             tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
             row.update({f"us{tag}": round(us, 2), f"tflops{tag}": round(tf, 1),
                         f"frac_of_peak{tag}": round(tf / peak, 4)})
+        # cuBLAS's block-scaled FP4 GEMM on the same operands (bf16 out), for reference
+        try:
+            import torch.nn.functional as F
+            A4 = ca.view(torch.float4_e2m1fn_x2)
+            B4 = cb.view(torch.float4_e2m1fn_x2).t()
+            s1 = ta.view(torch.float8_e8m0fnu).reshape(-1, K // 32)
+            s2 = tb.view(torch.float8_e8m0fnu).reshape(-1, K // 32)
+
+            def cublas():
+                return F.scaled_mm(A4, B4, s1, F.ScalingType.BlockWise1x32, s2, F.ScalingType.BlockWise1x32,
+                                   swizzle_a=F.SwizzleType.SWIZZLE_32_4_4,
+                                   swizzle_b=F.SwizzleType.SWIZZLE_32_4_4, output_dtype=torch.bfloat16)
+            for _ in range(W):
+                cublas()
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(K_launches):
+                cublas()
+            e1.record()
+            torch.cuda.synchronize(device)
+            us = e0.elapsed_time(e1) / K_launches * 1e3
+            tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            row.update({"us_cublas_mxfp4_bf16": round(us, 2), "tflops_cublas_mxfp4_bf16": round(tf, 1)})
+        except Exception as e:      # reference only
+            row["cublas_mxfp4"] = f"unavailable: {type(e).__name__}"
         out["shapes"][f"{M}x{N}x{K}"] = row
         del ca, cb, ta, tb, Y, Y16
     return out

@@ -207,3 +207,51 @@ def test_gemm_persistent_scaled_matches_oracle(kq, M, N, K):
     ref1 = o.gemm_mxfp4_rank1(ca[rows], sa[rows], cb, sb, mu[rows], wsum)
     tol1 = tol + 2.0 ** -22 * (np.abs(np.outer(mu[rows], wsum)) + np.abs(ref1))
     assert np.all(np.abs(Y1[rows] - ref1) <= tol1)
+
+
+# ---------------------------------------------------------------------------
+# the CTA-pair kernel (M, N multiples of 256, K of 256) on small shapes, and an
+# independent cross-check against cuBLAS's block-scaled FP4 GEMM
+# ---------------------------------------------------------------------------
+PAIR = [(256, 256, 256), (256, 512, 512), (768, 256, 1024), (512, 768, 2048)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR)
+def test_gemm_pair_kernel_matches_oracle(kq, M, N, K):
+    rng = np.random.default_rng(5 * M + N + K)
+    ca, sa = _operands(rng, M, K, 127, 127)
+    cb, sb = _operands(rng, N, K, 127, 127)
+    assert np.array_equal(_gemm(kq, ca, sa, cb, sb), o.gemm_mxfp4(ca, sa, cb, sb))
+    ca, sa = _operands(rng, M, K, 117, 137)
+    cb, sb = _operands(rng, N, K, 117, 137)
+    Y = _gemm(kq, ca, sa, cb, sb)
+    ref = o.gemm_mxfp4(ca, sa, cb, sb)
+    tol = (K / 64 + 64) * 2.0 ** -23 * o.gemm_error_scale(ca, sa, cb, sb)
+    assert np.all(np.abs(Y - ref) <= tol)
+    Y16 = _gemm_bf16(kq, ca, sa, cb, sb)
+    assert np.array_equal(_bf16_bits(Y16), _bf16_bits(torch.from_numpy(Y.astype(np.float32)).to(torch.bfloat16)))
+
+
+def test_gemm_matches_cublas_mxfp4(kq):
+    """cuBLAS's block-scaled FP4 GEMM (torch.nn.functional.scaled_mm with
+    E8M0 scales in the same 128 x 4 swizzled blocks) on the FLUX attention
+    projection: the same products in fp32, rounded to bf16, must give the
+    same bits (both the pair kernel and, at N = 3072 - 128, the single-CTA one)."""
+    F = pytest.importorskip("torch.nn.functional")
+    if not hasattr(F, "scaled_mm"):
+        pytest.skip("torch.nn.functional.scaled_mm not available")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    for M, N, K in ((4608, 3072, 3072), (4608, 2944, 3072)):
+        ca = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device="cuda", generator=g)
+        cb = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device="cuda", generator=g)
+        ta = kq.kq_sf_tile(torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device="cuda", generator=g))
+        tb = kq.kq_sf_tile(torch.randint(120, 134, (N, K // 32), dtype=torch.uint8, device="cuda", generator=g))
+        ours = kq.kq_gemm_mxfp4_bf16(ca, ta, cb, tb)
+        ref = F.scaled_mm(ca.view(torch.float4_e2m1fn_x2), cb.view(torch.float4_e2m1fn_x2).t(),
+                          ta.view(torch.float8_e8m0fnu).reshape(-1, K // 32), F.ScalingType.BlockWise1x32,
+                          tb.view(torch.float8_e8m0fnu).reshape(-1, K // 32), F.ScalingType.BlockWise1x32,
+                          swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                          output_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(ours.view(torch.int16), ref.view(torch.int16)), (M, N, K)

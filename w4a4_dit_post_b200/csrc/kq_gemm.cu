@@ -15,6 +15,10 @@
 // bytes, copied into all four lane quarters).  kq_sf_tile rewrites the
 // row-major scale bytes into such 512-byte blocks once per operand.
 //
+// Two kernels.  When M and N are multiples of 256 and K of 256, a cluster of
+// two CTAs computes 256 x 256 tiles with the pair MMA (gemm_pair_kernel,
+// below).  Otherwise the single-CTA kernel described here runs.
+//
 // Tiling.  Y is cut into 128 x 128 tiles; persistent CTAs (two per SM) walk
 // them.  Within a tile K advances in steps of 128
 // (64 bytes of codes per row, 4 scales): per step one TMA load of A and of B
@@ -439,6 +443,372 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair kernel: 256 x 256 output tiles over two SMs (cta_group::2)
+// ---------------------------------------------------------------------------
+// A cluster of two CTAs on two SMs computes one 256 x 256 tile of Y at a
+// time with the pair form of the block-scaled MMA: CTA r (r = 0, 1) holds rows
+// 128 r .. 128 r + 127 of the A tile and rows 128 r .. 128 r + 127 of the B
+// tile in its own shared memory, and each MMA (issued by CTA 0) reads A from
+// both CTAs and B from both CTAs, leaving rows 128 r .. of the 256 x 256
+// product in CTA r's tensor memory.  Every byte of A and B therefore crosses
+// from L2 once per pair instead of once per 128 x 128 tile: half the operand
+// traffic of the single-CTA kernel per FLOP.  The scales of a CTA's A rows
+// and of all 256 B rows are staged in each CTA and moved into its own tensor
+// memory by the pair copy.  No load uses cluster multicast: each CTA loads
+// only into its own shared memory; the loads of both CTAs complete on CTA 0's
+// barrier, and CTA 0's MMA completions arrive on both CTAs' barriers.
+//
+// A stage holds K = 256 (128-byte rows, 128-byte swizzle): per stage one
+// barrier round trip, six scale copies and four MMAs of K = 64.  With 64-byte
+// rows (K = 128, two MMAs a stage) the same kernel ran the 4608 x 3072 x 12288
+// layer no faster than the single-CTA kernel (117 against 108 us): the issue
+// of each stage, not operand bandwidth, was the limit.
+//
+// Roles (192 threads per CTA): warp 0 lane 0 loads (kPStages stages, in both
+// CTAs), warp 1 owns tensor memory (both CTAs) and, in CTA 0, lane 0 issues
+// the scale copies and the MMAs; warps 2..5 read the accumulator (one row per
+// thread), stage it in shared memory and write Y with TMA tensor stores.  One
+// accumulator of 256 columns: the epilogue hands it back as soon as it has
+// read it, before the stores.  Every wait is bounded; a wait that runs out
+// sets the device status word, the CTA drains, meets its peer at the final
+// cluster barrier and exits.
+constexpr int kPTile = 256;                        // tile rows and columns of a pair
+constexpr int kPHalf = 128;                        // rows of A and of B in each CTA
+constexpr int kPK = 256;                           // K per stage (fp4 elements): 128-byte rows
+constexpr int kPKb = kPK / 128;                    // 128-K scale blocks per stage
+constexpr int kPStages = 4;
+constexpr int kPOpBytes = kPHalf * kPK / 2;        // codes per operand per stage
+constexpr int kPStageTx = 2 * kPOpBytes + 3 * kPKb * kSfBytes;   // bytes one CTA loads per stage
+constexpr int kPStageBytes = (kPStageTx + 1023) & ~1023;         // a multiple of 1 KiB
+constexpr int kPOutBytes = 4 * kPHalf * 128;       // four [128 rows][128 B] staging chunks
+constexpr int kPTmemCols = 512;
+// after the 256 accumulator columns: A scales (4 columns per 128-K block),
+// then B scales (8 columns per 128-K block: 4 for each 128 rows of the 256)
+constexpr int kPSfaCol = 256, kPSfbCol = 256 + 4 * kPKb;
+static_assert(kPSfbCol + 8 * kPKb <= kPTmemCols, "tensor memory layout");
+
+// Shared-memory descriptor of a K-major operand tile whose rows are 128 bytes
+// (K = 256 fp4), 128-byte swizzle: 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+
+
+__host__ __device__ constexpr int pair_smem_bytes() {
+  return 1024 + kPStages * kPStageBytes + kPOutBytes + 256;
+}
+
+// M = 256 (the pair), N = 256, K = 64, E2M1 x E2M1, E8M0 scales, K-major.
+constexpr uint32_t kPIdescBase = (1u << 7) | (1u << 10) | ((uint32_t)(kPTile >> 3) << 17) | (1u << 23) |
+                                 ((uint32_t)(kPTile >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// 2-D TMA load into this CTA's shared memory whose completion is counted on a
+// barrier of CTA 0 of the pair (`bar` is that barrier's cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, int c0, int c1,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Scale block from each CTA's shared memory into its own tensor memory.
+__device__ __forceinline__ void sf_copy_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair once the
+// MMAs issued so far have completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\t"
+      "mov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}"
+      ::"r"(bar)
+      : "memory");
+}
+
+struct PairArgs {
+  int M, N;
+  int k_steps;               // K / 128
+  int m_tiles, n_tiles;      // 256-row and 256-column tiles
+  int pairs;                 // clusters in the grid
+};
+
+// Bounded wait for a time well above any in-flight copy or MMA, used only on
+// the abort path before the CTA leaves (nothing else tells it when the
+// peer's copies into its shared memory have landed).
+__device__ __forceinline__ void settle_ns(uint64_t ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < ns) {}
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                 const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
+                 const __grid_constant__ CUtensorMap ymap, const PairArgs args, unsigned int* devstat) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* out_stage = smem + kPStages * kPStageBytes;           // 4 x [128 rows][128 B], 128B swizzle
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + kPOutBytes);
+  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kPStages]);
+  const uint32_t accf = smem_addr(&bars[2 * kPStages]), acce = smem_addr(&bars[2 * kPStages + 1]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kPStages + 2]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kPStages + 3]);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();              // 0: issues the MMAs
+  const int pair = (int)blockIdx.x >> 1;
+  const int KS = args.k_steps;             // stages of K per tile
+  const int KS128 = KS * kPKb;             // 128-K scale blocks per row block
+  const int n_tiles_total = args.m_tiles * args.n_tiles;
+  const int my_tiles = pair < n_tiles_total ? (n_tiles_total - pair + args.pairs - 1) / args.pairs : 0;
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&bmap);
+    tma_prefetch_desc(&sfamap);
+    tma_prefetch_desc(&sfbmap);
+    tma_prefetch_desc(&ymap);
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accf, 1);
+    mbar_init(acce, 2 * (kEpiThreads / 32));        // every epilogue warp of both CTAs
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kPTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  // both CTAs' barriers are initialised before any copy or commit targets them
+  cluster_sync_all();
+  fence_after_sync();
+  pdl_wait_predecessor();
+  const uint32_t tmem_base = *tmem_slot;
+  bool aborted = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int seq = 0;
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+        const int t = pair + i * args.pairs;
+        const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
+        const int arow = m_tile * kPTile + (int)rank * kPHalf;
+        const int brow = n_tile * kPTile + (int)rank * kPHalf;
+        const int sfa_blk = (m_tile * 2 + (int)rank) * KS128, sfb_blk = n_tile * 2 * KS128;
+        for (int kt = 0; kt < KS; ++kt, ++seq) {
+          const int s = seq % kPStages;
+          if (seq >= kPStages && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(seq / kPStages - 1) & 1u)) {
+            *abort_flag = 1;
+            atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+            break;
+          }
+          const uint32_t st = smem_addr(smem + s * kPStageBytes);
+          const uint32_t bar = map_to_rank(full0 + 8 * s, 0);
+          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)(2 * kPStageTx));
+          // codes, then the scale blocks of this stage's kPKb 128-K blocks: A's
+          // rows, then the first and the second 128 rows of B
+          tma_load_2d_pair(st, &amap, kt * (kPK / 2), arow, bar);
+          tma_load_2d_pair(st + kPOpBytes, &bmap, kt * (kPK / 2), brow, bar);
+          const uint32_t sf = st + 2 * kPOpBytes;
+          tma_load_2d_pair(sf, &sfamap, 0, sfa_blk + kPKb * kt, bar);
+          tma_load_2d_pair(sf + kPKb * kSfBytes, &sfbmap, 0, sfb_blk + kPKb * kt, bar);
+          tma_load_2d_pair(sf + 2 * kPKb * kSfBytes, &sfbmap, 0, sfb_blk + KS128 + kPKb * kt, bar);
+        }
+      }
+      aborted = *abort_flag != 0;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      int seq = 0;
+      for (int i = 0; i < my_tiles; ++i) {
+        // both CTAs' epilogues have read the previous tile's accumulator
+        bool ok = i == 0 || mbar_wait_bounded(acce, (uint32_t)(i - 1) & 1u);
+        if (ok) fence_after_sync();
+        for (int kt = 0; ok && kt < KS; ++kt, ++seq) {
+          const int s = seq % kPStages;
+          ok = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(seq / kPStages) & 1u) && !*abort_flag;
+          if (!ok) break;
+          fence_after_sync();
+          const uint32_t st = smem_addr(smem + s * kPStageBytes);
+          const uint32_t sf = st + 2 * kPOpBytes;
+#pragma unroll
+          for (int j = 0; j < kPKb; ++j) {
+            sf_copy_pair(tmem_base + kPSfaCol + 4 * j, sf_desc(sf + j * kSfBytes));
+            sf_copy_pair(tmem_base + kPSfbCol + 8 * j, sf_desc(sf + (kPKb + j) * kSfBytes));
+            sf_copy_pair(tmem_base + kPSfbCol + 8 * j + 4, sf_desc(sf + (2 * kPKb + j) * kSfBytes));
+          }
+          // K = 64 per MMA: MMA kk reads scale block kk / 2, scales 2 (kk % 2) and 2 (kk % 2) + 1
+#pragma unroll
+          for (int kk = 0; kk < 2 * kPKb; ++kk) {
+            const int j = kk >> 1;
+            const uint32_t sf_id = (uint32_t)(2 * (kk & 1));
+            const uint32_t sfa = (tmem_base + kPSfaCol + 4 * j) | (sf_id << 30);
+            const uint32_t sfb = (tmem_base + kPSfbCol + 8 * j) | (sf_id << 30);
+            const uint32_t idesc = kPIdescBase | (sf_id << 29) | (sf_id << 4);
+            mma_mxf4_pair(tmem_base, sw128_desc(st + kk * 32), sw128_desc(st + kPOpBytes + kk * 32),
+                          idesc, sfa, sfb, (kt | kk) != 0);
+          }
+          mma_commit_pair(empty0 + 8 * s);
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+          break;
+        }
+        mma_commit_pair(accf);
+      }
+      aborted = *abort_flag != 0;
+    }
+  } else {
+    // epilogue: warps 2..5 -> tensor-memory lane quarters (warp % 4); thread = one row
+    const int q = warp & 3;
+    const int etid = tid - 64;
+    const int r_local = 32 * q + lane;
+    const uint32_t acce_leader = map_to_rank(acce, 0);
+    for (int i = 0; i < my_tiles; ++i) {
+      const int t = pair + i * args.pairs;
+      const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
+      const int row0 = m_tile * kPTile + (int)rank * kPHalf, n0 = n_tile * kPTile;
+      const bool ok = mbar_wait_bounded(accf, (uint32_t)i & 1u);
+      // the previous tile's stores have read the staging chunks
+      if (etid == 0) bulk_wait_read_all();
+      if (epi_any(!ok || *abort_flag)) {
+        if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
+        *abort_flag = 1;
+        aborted = true;
+        break;
+      }
+      fence_after_sync();
+      if constexpr (kBf16) {
+        // all 256 columns, as bf16, into the four chunks (64 columns = 128 B a row each)
+        for (int c = 0; c < kPTile / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+          uint32_t w[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const __nv_bfloat162 h2 =
+                __floats2bfloat162_rn(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+            w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          if (c == kPTile / 32 - 1) {
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acce_leader);
+          }
+          uint8_t* rowp = out_stage + (c >> 1) * (kPHalf * 128) + r_local * 128;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = (c & 1) * 4 + u;
+            *reinterpret_cast<uint4*>(rowp + ((j ^ (r_local & 7)) << 4)) =
+                make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        epi_barrier();
+        if (etid == 0) {
+          for (int h = 0; h < 4; ++h)
+            tma_store_2d(&ymap, n0 + 64 * h, row0, smem_addr(out_stage + h * (kPHalf * 128)));
+          bulk_commit();
+        }
+      } else {
+        // fp32: two halves of 128 columns (four chunks of 32 columns each)
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1) {
+            if (etid == 0) bulk_wait_read_all();
+            epi_barrier();
+          }
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * h + 32 * c), r);
+            if (h == 1 && c == 3) {
+              fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_remote(acce_leader);
+            }
+            uint8_t* rowp = out_stage + c * (kPHalf * 128) + r_local * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(rowp + ((u ^ (r_local & 7)) << 4)) =
+                  make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          epi_barrier();
+          if (etid == 0) {
+            for (int c = 0; c < 4; ++c)
+              tma_store_2d(&ymap, n0 + 128 * h + 32 * c, row0, smem_addr(out_stage + c * (kPHalf * 128)));
+            bulk_commit();
+          }
+        }
+      }
+    }
+    if (etid == 0) bulk_wait_all();
+  }
+
+  // Leave together: after a timeout, give copies and MMAs already in flight
+  // (microseconds of work) time to land first; then every thread of both
+  // CTAs meets at the cluster barrier, so no CTA exits while its peer may
+  // still reach its shared or tensor memory.
+  if (__syncthreads_or(aborted)) settle_ns(20000000ull);
+  fence_before_sync();
+  cluster_sync_all();
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kPTmemCols)
+                 : "memory");
+  }
+}
+
 // Row-major scale bytes [R][K/32] -> 512-byte blocks [ceil(R/128)][K/128][512]
 // (row r, scale column s at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + s % 4
 // of block (r / 128, s / 4)); rows past R become zero.  One thread per output byte.
@@ -487,6 +857,102 @@ int codes_tmap(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t K) {
 }
 
 constexpr int kMaxDevices = 64;
+
+// Tiled scale blocks [rows / 128 * K / 128][512 bytes] seen as a 2-D tensor of
+// 128 32-bit words per block; one box is one 512-byte block.
+int sf_tmap(CUtensorMap* tm, const uint8_t* tiled, int64_t rows, int64_t K) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = gemm_encoder();
+  if (!enc) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled not found in the CUDA driver");
+  const cuuint64_t dims[2] = {128, (cuuint64_t)((rows + 127) / 128 * (K / 128))};
+  const cuuint64_t strides[1] = {512};
+  const cuuint32_t box[2] = {128, (cuuint32_t)gemm::kPKb};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(tiled), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (CUresult %d)", (int)r);
+  return KQ_OK;
+}
+
+// Codes [rows][K/2] for the pair kernel: box 128 bytes (K = 256) x 128 rows,
+// 128-byte swizzle (the canonical K-major layout of 128-byte rows).
+int pair_codes_tmap(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t K) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = gemm_encoder();
+  if (!enc) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled not found in the CUDA driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+  const cuuint32_t box[2] = {gemm::kPK / 2, gemm::kPHalf};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return KQ_OK;
+}
+
+// The CTA-pair kernel for M and N multiples of 256 and K a multiple of the
+// stage's K (no rank-1 term).
+int gemm_pair_launch(const uint8_t* a_codes, const uint8_t* b_codes, const CUtensorMap& ym,
+                     const uint8_t* a_sf_tiled, const uint8_t* b_sf_tiled, int64_t M, int64_t N,
+                     int64_t K, bool bf16, unsigned int* devstat, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  const int smem = gemm::pair_smem_bytes();
+  static std::once_flag attr_once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  std::call_once(attr_once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(gemm::gemm_pair_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (attr_err[dev] == cudaSuccess)
+      attr_err[dev] = cudaFuncSetAttribute(gemm::gemm_pair_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute (pair)");
+
+  CUtensorMap am, bm, sam, sbm;
+  if (int st = pair_codes_tmap(&am, a_codes, M, K)) return st;
+  if (int st = pair_codes_tmap(&bm, b_codes, N, K)) return st;
+  if (int st = sf_tmap(&sam, a_sf_tiled, M, K)) return st;
+  if (int st = sf_tmap(&sbm, b_sf_tiled, N, K)) return st;
+  gemm::PairArgs args;
+  args.M = (int)M;
+  args.N = (int)N;
+  args.k_steps = (int)(K / gemm::kPK);
+  args.m_tiles = (int)(M / gemm::kPTile);
+  args.n_tiles = (int)(N / gemm::kPTile);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(gemm::kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  auto kern = bf16 ? gemm::gemm_pair_kernel<true> : gemm::gemm_pair_kernel<false>;
+  // as many pairs as can be resident at once (one CTA per SM), no more than tiles
+  int sms = 0;
+  if (int st = sm_count(&sms)) return st;
+  cfg.gridDim = dim3((unsigned)sms);
+  int clusters = 0;
+  err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaOccupancyMaxActiveClusters");
+  if (clusters < 1) return fail(KQ_ERR_UNSUPPORTED, "gemm: no CTA pair fits on the device");
+  const int64_t tiles = (int64_t)args.m_tiles * args.n_tiles;
+  if (clusters > tiles) clusters = (int)tiles;
+  args.pairs = clusters;
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  err = cudaLaunchKernelEx(&cfg, kern, am, bm, sam, sbm, ym, args, devstat);
+  if (err != cudaSuccess) return cuda_fail(err, "gemm_pair_kernel launch");
+  return check_launch("gemm_pair_kernel launch");
+}
 
 }  // namespace
 }  // namespace kq
@@ -550,6 +1016,12 @@ int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t
                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return kq::fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed (CUresult %d)", (int)r);
   }
+  unsigned int* devstat = nullptr;
+  if (int st = kq::device_status_address(&devstat)) return st;
+  if (M % kq::gemm::kPTile == 0 && N % kq::gemm::kPTile == 0 && K % kq::gemm::kPK == 0 &&
+      mu == nullptr && tma_store)
+    return kq::gemm_pair_launch(a_codes, b_codes, ym, a_sf_tiled, b_sf_tiled, M, N, K, bf16, devstat,
+                                kq::as_stream(stream));
   kq::gemm::GemmArgs args;
   args.M = (int)M;
   args.N = (int)N;
@@ -563,8 +1035,6 @@ int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t
   args.n_tiles = (int)((N + 127) / 128);
   args.mu = mu;
   args.wsum = wsum;
-  unsigned int* devstat = nullptr;
-  if (int st = kq::device_status_address(&devstat)) return st;
 
   cudaLaunchConfig_t cfg = {};
   int sms = 0;
