@@ -266,7 +266,7 @@ def test_expand_params(kq):
     assert np.all(np.abs(T - T_ref) <= 1e-6 * mag)
 
 
-@pytest.mark.parametrize("N,d", [(1, 32), (24, 128), (384, 1152), (3072, 3072)])
+@pytest.mark.parametrize("N,d", [(1, 32), (24, 128), (384, 1152), (5, 3072), (7, 12288), (3072, 3072)])
 def test_fold_weights(kq, N, d):
     p, pd = params_dev(d // 32, 41)
     W = synthetic.make_weights(N, d, 5)

@@ -1,7 +1,7 @@
 // Support kernels: the dense blocks of the transform (kq_expand_params), the
 // inverse folded into the weights (kq_fold_weights), the folded weights
-// quantised to MXFP4 (kq_quantize_weights) and MXFP4 decoding (kq_dequant).  None of them is on the per-step path; they are simple,
-// memory-bound grid-stride kernels.
+// quantised to MXFP4 (kq_quantize_weights) and MXFP4 decoding (kq_dequant).
+// None of them is on the per-step path; they are memory-bound kernels.
 #include <cuda_runtime.h>
 
 #include "kq.h"
@@ -35,41 +35,93 @@ expand_kernel(const float* __restrict__ params, int nb, float* __restrict__ T, u
   }
 }
 
-// One thread per (weight row, 32-column block): w <- w T_j^{-1}, applied as the
-// butterfly of the transposed inverse factors.  Reads the whole block before
-// writing it, so in-place use is safe.
+// The fold with coalesced traffic: a warp takes 32 consecutive blocks (4 KiB
+// of W), reads them with 16-byte loads into shared memory (chunk c of block b
+// at c ^ (b % 8): conflict-free both ways), each lane folds its own block and
+// puts it back in the same slots, and the warp writes the 4 KiB with 16-byte
+// stores.  The warp has read its whole piece before it writes any of it, and
+// warps own disjoint pieces, so in-place use stays safe.  kCS (nb a multiple
+// of 32): the warp keeps one 32-block column group and walks the rows, so
+// each lane builds its five transposed inverse factors once; otherwise every
+// block loads its own parameters.
+template <bool kCS>
 __global__ void __launch_bounds__(kAuxThreads)
-fold_kernel(const float* W, const float* __restrict__ params, int nb, int n_blocks, float* W_out,
-            unsigned int* devstat) {
-  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n_blocks; g += gridDim.x * blockDim.x) {
-    const int j = g % nb;
+fold_coalesced_kernel(const float* W, const float* __restrict__ params, int N, int nb, int n_blocks,
+                      float* W_out, unsigned int* devstat) {
+  __shared__ float4 stage[kAuxThreads / 32][32 * 8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4* st = stage[warp];
+  const int warps_total = gridDim.x * (blockDim.x >> 5);
+  const int wglob = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int n_cg = nb / 32;
+  float4 B[5];
+  if constexpr (kCS) {
+    // warps past the last whole round of column groups would repeat pieces
+    // of the warps below them (harmful in place): they leave
+    if (wglob >= (warps_total / n_cg) * n_cg) return;      // warp-uniform
+    const int j = (wglob % n_cg) * 32 + lane;
     const float* p = params + 15 * j;
-    float4 B[5];
     bool bad = false;
 #pragma unroll
     for (int m = 0; m < 5; ++m) {
       bad |= lu_params_bad(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
       B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
     }
-    if (bad && g < nb) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
-    const float4* src = reinterpret_cast<const float4*>(W + (size_t)g * 32);
-    float2 v[16];
+    if (bad && wglob < n_cg) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
+  }
+  // piece u: kCS -> row u / n_cg, column group u % n_cg (the step keeps the
+  // group); otherwise blocks 32 u .. 32 u + 31 of the flattened weight
+  const int n_pieces = kCS ? N * n_cg : (n_blocks + 31) / 32;
+  const int step = kCS ? (warps_total / n_cg) * n_cg : warps_total;
+  for (int u = wglob; u < n_pieces; u += step) {
+    const size_t g0 = kCS ? (size_t)(u / n_cg) * nb + (size_t)(u % n_cg) * 32 : (size_t)u * 32;
+    const int nblk = kCS ? 32 : (n_blocks - (int)g0 < 32 ? n_blocks - (int)g0 : 32);
+    const float4* src = reinterpret_cast<const float4*>(W + g0 * 32);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 t = src[q];
-      v[2 * q] = make_float2(t.x, t.y);
-      v[2 * q + 1] = make_float2(t.z, t.w);
+    for (int i = 0; i < 8; ++i) {
+      const int L = lane + 32 * i;            // 16-byte chunk of the warp's 4 KiB
+      const int b = L >> 3, c = L & 7;
+      if (kCS || L < nblk * 8) st[b * 8 + (c ^ (b & 7))] = src[L];
     }
-    butterfly32(v, B);
-    float4* dst = reinterpret_cast<float4*>(W_out + (size_t)g * 32);
+    __syncwarp();
+    if (kCS || lane < nblk) {
+      if constexpr (!kCS) {
+        const int g = (int)g0 + lane;
+        const float* p = params + 15 * (g % nb);
+        bool bad = false;
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      dst[q] = make_float4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
+        for (int m = 0; m < 5; ++m) {
+          bad |= lu_params_bad(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+          B[m] = lu_factor_inv_t(p[3 * m], p[3 * m + 1], p[3 * m + 2]);
+        }
+        if (bad && g < nb) atomicOr(devstat, (unsigned)KQ_DEVSTAT_BAD_PARAMS);
+      }
+      float2 v[16];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 t = st[lane * 8 + (q ^ (lane & 7))];
+        v[2 * q] = make_float2(t.x, t.y);
+        v[2 * q + 1] = make_float2(t.z, t.w);
+      }
+      butterfly32(v, B);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st[lane * 8 + (q ^ (lane & 7))] = make_float4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
+    }
+    __syncwarp();
+    float4* dst = reinterpret_cast<float4*>(W_out + g0 * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int L = lane + 32 * i;
+      const int b = L >> 3, c = L & 7;
+      if (kCS || L < nblk * 8) dst[L] = st[b * 8 + (c ^ (b & 7))];
+    }
+    __syncwarp();
   }
 }
 
 // Weight side: one thread per (weight row, block): the folded block
-// w T_j^{-1} (the same butterfly as fold_kernel) encoded to MXFP4 in
+// w T_j^{-1} (the same butterfly as fold_coalesced_kernel) encoded to MXFP4 in
 // registers; the folded weights are never written.  A warp takes 32
 // consecutive blocks (4 KiB of W): it reads them with coalesced 16-byte loads
 // into shared memory (16-byte chunk c of block b stored at chunk c ^ (b % 8),
@@ -292,9 +344,27 @@ int kq_fold_weights(const float* W, int64_t N, int64_t d, const float* params, f
   const int n_blocks = (int)(N * nb);
   unsigned int* devstat = nullptr;
   if (int st = kq::device_status_address(&devstat)) return st;
-  kq::fold_kernel<<<kq::grid_for(n_blocks), kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
-      W, params, nb, n_blocks, W_out, devstat);
-  return kq::check_launch("fold_kernel launch");
+  int sms = 0;
+  if (int st = kq::sm_count(&sms)) return st;
+  const int warps_per_cta = kq::kAuxThreads / 32;
+  if (nb % 32 == 0) {
+    // a whole number of warps per column group, enough to fill the device
+    const int n_cg = nb / 32;
+    int64_t groups_per_cg = (int64_t)sms * 8 * warps_per_cta / n_cg;
+    if (groups_per_cg > N) groups_per_cg = N;
+    if (groups_per_cg < 1) groups_per_cg = 1;
+    int64_t warps = groups_per_cg * n_cg;
+    const int64_t ctas = (warps + warps_per_cta - 1) / warps_per_cta;   // >= n_cg warps
+    kq::fold_coalesced_kernel<true><<<(unsigned)ctas, kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+        W, params, (int)N, nb, n_blocks, W_out, devstat);
+  } else {
+    const int pieces = (n_blocks + 31) / 32;
+    int ctas = (pieces + warps_per_cta - 1) / warps_per_cta;
+    if (ctas > sms * 8) ctas = sms * 8;
+    kq::fold_coalesced_kernel<false><<<(unsigned)ctas, kq::kAuxThreads, 0, kq::as_stream(stream)>>>(
+        W, params, (int)N, nb, n_blocks, W_out, devstat);
+  }
+  return kq::check_launch("fold_coalesced_kernel launch");
 }
 
 int kq_quantize_weights(const float* W, int64_t N, int64_t d, const float* params,
