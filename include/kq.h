@@ -218,10 +218,10 @@ int kq_sf_tile(const uint8_t* scales, int64_t R, int64_t K, uint8_t* tiled, void
  *   [M][K/2] from kq_quantize, scales tiled by kq_sf_tile), b = the MXFP4
  *   folded weights (codes [N][K/2] from kq_quantize_weights, scales tiled).
  *   Y [M][N] fp32 row-major.  Products on the tensor cores with the
- *   block-scaled FP4 MMA, fp32 accumulation in tensor memory.  When M and N
- *   are multiples of 256 and K of 256 the work runs on pairs of SMs (256 x 256
- *   tiles, one MMA over both SMs' shared memory); the result does not depend
- *   on which kernel ran.
+ *   block-scaled FP4 MMA, fp32 accumulation in tensor memory.  When M and K
+ *   are multiples of 256 and N of 256 (or else of 192) the work runs on pairs
+ *   of SMs (256 x 256 or 256 x 192 tiles, one MMA over both SMs' shared
+ *   memory); the result does not depend on which kernel ran.
  *   K a multiple of 128; all pointers 16-byte aligned; M, N < 2^31.
  */
 int kq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t* b_codes,

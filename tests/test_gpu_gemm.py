@@ -157,11 +157,14 @@ def test_quantize_with_tiled_scales(kq, M, d):
 
 
 # ---------------------------------------------------------------------------
-# the persistent schedule: more 128 x 128 output tiles than CTAs (two per SM
-# on 148 SMs = 296), so every CTA walks two or more tiles and the stage ring
-# and the accumulator hand-back carry over from one tile to the next
+# the persistent schedule: more output tiles than CTAs or CTA pairs, so they
+# walk two or more tiles and the stage ring and the accumulator hand-back
+# carry over from one tile to the next.  2176 x 2304: the single-CTA kernel,
+# 306 tiles of 128 x 128 over 296 CTAs; 2048 x 2560 and 4608 x 3072: the pair
+# kernel, 80 and 216 tiles of 256 x 256 over 74 pairs; 4608 x 2880: 270
+# tiles of 256 x 192 (two accumulators)
 # ---------------------------------------------------------------------------
-MULTI_TILE = [(2048, 2560, 1024), (2176, 2304, 512), (4608, 3072, 3072)]   # 320, 306, 864 tiles
+MULTI_TILE = [(2048, 2560, 1024), (2176, 2304, 512), (4608, 3072, 3072), (4608, 2880, 1024)]
 
 
 def _sampled_rows(M, n, seed):
@@ -210,10 +213,16 @@ def test_gemm_persistent_scaled_matches_oracle(kq, M, N, K):
 
 
 # ---------------------------------------------------------------------------
-# the CTA-pair kernel (M, N multiples of 256, K of 256) on small shapes, and an
-# independent cross-check against cuBLAS's block-scaled FP4 GEMM
+# the CTA-pair kernel (M and K multiples of 256; N a multiple of 256: 256 x 256
+# tiles and one accumulator, else of 192: 256 x 192 tiles and two) on small
+# shapes, and an independent cross-check against cuBLAS's block-scaled FP4
+# GEMM.  192-wide tiles with odd indices read B scales from the middle of a
+# 128-row scale block.  2560 x 3840 has 150 tiles and 2560 x 2880 has 150
+# (192-wide), so some pairs run three tiles: the accumulator barriers turn
+# over.
 # ---------------------------------------------------------------------------
-PAIR = [(256, 256, 256), (256, 512, 512), (768, 256, 1024), (512, 768, 2048)]
+PAIR = [(256, 256, 256), (256, 512, 512), (768, 256, 1024), (512, 768, 2048), (2560, 3840, 512),  # 256 wide
+        (256, 192, 256), (512, 576, 512), (768, 1344, 1024), (2560, 2880, 512)]                   # 192 wide
 
 
 @pytest.mark.parametrize("M,N,K", PAIR)
@@ -236,13 +245,14 @@ def test_gemm_matches_cublas_mxfp4(kq):
     """cuBLAS's block-scaled FP4 GEMM (torch.nn.functional.scaled_mm with
     E8M0 scales in the same 128 x 4 swizzled blocks) on the FLUX attention
     projection: the same products in fp32, rounded to bf16, must give the
-    same bits (both the pair kernel and, at N = 3072 - 128, the single-CTA one)."""
+    same bits (the pair kernel with 192- and 256-column tiles and, at
+    N = 3072 - 128, the single-CTA one)."""
     F = pytest.importorskip("torch.nn.functional")
     if not hasattr(F, "scaled_mm"):
         pytest.skip("torch.nn.functional.scaled_mm not available")
     g = torch.Generator(device="cuda")
     g.manual_seed(11)
-    for M, N, K in ((4608, 3072, 3072), (4608, 2944, 3072)):
+    for M, N, K in ((4608, 3072, 3072), (4608, 2880, 3072), (4608, 2944, 3072)):
         ca = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device="cuda", generator=g)
         cb = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device="cuda", generator=g)
         ta = kq.kq_sf_tile(torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device="cuda", generator=g))

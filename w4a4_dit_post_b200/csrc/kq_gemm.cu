@@ -15,9 +15,10 @@
 // bytes, copied into all four lane quarters).  kq_sf_tile rewrites the
 // row-major scale bytes into such 512-byte blocks once per operand.
 //
-// Two kernels.  When M and N are multiples of 256 and K of 256, a cluster of
-// two CTAs computes 256 x 256 tiles with the pair MMA (gemm_pair_kernel,
-// below).  Otherwise the single-CTA kernel described here runs.
+// Two kernels.  When M and K are multiples of 256 and N of 192 or 256, a
+// cluster of two CTAs computes 256 x 192 or 256 x 256 tiles with the pair MMA
+// (gemm_pair_kernel, below).  Otherwise the single-CTA kernel described here
+// runs.
 //
 // Tiling.  Y is cut into 128 x 128 tiles; persistent CTAs (two per SM) walk
 // them.  Within a tile K advances in steps of 128
@@ -117,12 +118,12 @@ __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void epi_barrier() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+__device__ __forceinline__ void epi_barrier(int threads = kEpiThreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
 }
 // Barrier 1 among the epilogue warps that also ORs a flag across them, so
 // that all of them take the same branch (none is left at a barrier).
-__device__ __forceinline__ bool epi_any(bool pred) {
+__device__ __forceinline__ bool epi_any(bool pred, int threads = kEpiThreads) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
@@ -130,7 +131,7 @@ __device__ __forceinline__ bool epi_any(bool pred) {
       "bar.red.or.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred), "r"(kEpiThreads)
+      : "r"((uint32_t)pred), "r"(threads)
       : "memory");
   return r != 0;
 }
@@ -155,6 +156,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+// 32 consecutive fp32 accumulator columns of this thread's lane; the
+// registers are valid only after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20,"
+      "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 struct GemmArgs {
   int M, N, K;
@@ -444,20 +461,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
 }
 
 // ---------------------------------------------------------------------------
-// CTA-pair kernel: 256 x 256 output tiles over two SMs (cta_group::2)
+// CTA-pair kernel: 256 x kTN output tiles over two SMs (cta_group::2)
 // ---------------------------------------------------------------------------
-// A cluster of two CTAs on two SMs computes one 256 x 256 tile of Y at a
+// A cluster of two CTAs on two SMs computes one 256 x kTN tile of Y at a
 // time with the pair form of the block-scaled MMA: CTA r (r = 0, 1) holds rows
-// 128 r .. 128 r + 127 of the A tile and rows 128 r .. 128 r + 127 of the B
-// tile in its own shared memory, and each MMA (issued by CTA 0) reads A from
-// both CTAs and B from both CTAs, leaving rows 128 r .. of the 256 x 256
+// 128 r .. 128 r + 127 of the A tile and rows r kTN/2 .. (r + 1) kTN/2 - 1 of
+// the B tile in its own shared memory, and each MMA (issued by CTA 0) reads A
+// from both CTAs and B from both CTAs, leaving rows 128 r .. of the 256 x kTN
 // product in CTA r's tensor memory.  Every byte of A and B therefore crosses
-// from L2 once per pair instead of once per 128 x 128 tile: half the operand
-// traffic of the single-CTA kernel per FLOP.  The scales of a CTA's A rows
-// and of all 256 B rows are staged in each CTA and moved into its own tensor
-// memory by the pair copy.  No load uses cluster multicast: each CTA loads
-// only into its own shared memory; the loads of both CTAs complete on CTA 0's
-// barrier, and CTA 0's MMA completions arrive on both CTAs' barriers.
+// from L2 once per pair instead of once per 128-row tile: half the operand
+// traffic of the single-CTA kernel per FLOP.  The scales of a CTA's A rows and
+// of the B rows of the tile are staged in each CTA and moved into its own
+// tensor memory by the pair copy.  No load uses cluster multicast: each CTA
+// loads only into its own shared memory; the loads of both CTAs complete on
+// CTA 0's barrier, and CTA 0's MMA completions arrive on both CTAs' barriers.
+//
+// Tile width.  kTN = 192 (N a multiple of 192): two accumulators of 192
+// columns fit in tensor memory beside the scales, so the MMAs of the next tile
+// run while the epilogue drains the last one.  kTN = 256 (other N, multiples
+// of 256): one accumulator of 256 columns (two would leave no column for the
+// scales), handed back as soon as the epilogue has read it, before the
+// stores.  Scale blocks cover 128 B rows; a 192-column tile with an odd index
+// starts half-way through one, so it loads the two blocks it meets and points
+// the MMA's B-scale address two tensor-memory columns (64 rows) in.
 //
 // A stage holds K = 256 (128-byte rows, 128-byte swizzle): per stage one
 // barrier round trip, six scale copies and four MMAs of K = 64.  With 64-byte
@@ -465,28 +491,43 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
 // layer no faster than the single-CTA kernel (117 against 108 us): the issue
 // of each stage, not operand bandwidth, was the limit.
 //
-// Roles (192 threads per CTA): warp 0 lane 0 loads (kPStages stages, in both
-// CTAs), warp 1 owns tensor memory (both CTAs) and, in CTA 0, lane 0 issues
-// the scale copies and the MMAs; warps 2..5 read the accumulator (one row per
-// thread), stage it in shared memory and write Y with TMA tensor stores.  One
-// accumulator of 256 columns: the epilogue hands it back as soon as it has
-// read it, before the stores.  Every wait is bounded; a wait that runs out
-// sets the device status word, the CTA drains, meets its peer at the final
-// cluster barrier and exits.
-constexpr int kPTile = 256;                        // tile rows and columns of a pair
-constexpr int kPHalf = 128;                        // rows of A and of B in each CTA
+// Roles (320 threads per CTA): warp 0 lane 0 loads (in both CTAs), warp 1
+// owns tensor memory (both CTAs) and, in CTA 0, lane 0 issues the scale
+// copies and the MMAs; warps 2..9 read the accumulator (two warps per lane
+// quarter, one row per thread, half of the columns each, in one round trip),
+// hand it back, stage Y in shared memory and write it with TMA tensor stores.  Every wait is
+// bounded; a wait that runs out sets the device status word, the CTA drains,
+// meets its peer at the final cluster barrier and exits.
+constexpr int kPM = 256;                           // tile rows of a pair (the MMA's M)
+constexpr int kPHalf = 128;                        // rows of A in each CTA
 constexpr int kPK = 256;                           // K per stage (fp4 elements): 128-byte rows
 constexpr int kPKb = kPK / 128;                    // 128-K scale blocks per stage
-constexpr int kPStages = 4;
-constexpr int kPOpBytes = kPHalf * kPK / 2;        // codes per operand per stage
-constexpr int kPStageTx = 2 * kPOpBytes + 3 * kPKb * kSfBytes;   // bytes one CTA loads per stage
-constexpr int kPStageBytes = (kPStageTx + 1023) & ~1023;         // a multiple of 1 KiB
-constexpr int kPOutBytes = 4 * kPHalf * 128;       // four [128 rows][128 B] staging chunks
+constexpr int kPOpBytes = kPHalf * kPK / 2;        // A codes per CTA per stage
 constexpr int kPTmemCols = 512;
-// after the 256 accumulator columns: A scales (4 columns per 128-K block),
-// then B scales (8 columns per 128-K block: 4 for each 128 rows of the 256)
-constexpr int kPSfaCol = 256, kPSfbCol = 256 + 4 * kPKb;
-static_assert(kPSfbCol + 8 * kPKb <= kPTmemCols, "tensor memory layout");
+constexpr int kPAccStride = 256;                   // tensor-memory columns between accumulators
+
+template <int kTN>
+struct PairShape {
+  static_assert(kTN == 192 || kTN == 256, "pair tile width");
+  static constexpr int kBHalf = kTN / 2;                        // rows of B in each CTA
+  static constexpr int kBufs = kTN == 256 ? 1 : 2;              // accumulators
+  static constexpr int kStages = kTN == 256 ? 4 : 5;
+  static constexpr int kOutChunks = 4;                          // [128 rows][128 B] staging chunks
+  static constexpr int kBBytes = kBHalf * kPK / 2;              // B codes per CTA per stage
+  // bytes one CTA loads per stage: codes, A's scale blocks, two blocks of B scales
+  static constexpr int kStageTx = kPOpBytes + kBBytes + 3 * kPKb * kSfBytes;
+  static constexpr int kStageBytes = (kStageTx + 1023) & ~1023;   // a multiple of 1 KiB
+  // after the accumulators: A scales (4 columns per 128-K block), then B
+  // scales (8 columns per 128-K block: two 128-row blocks)
+  static constexpr int kSfaCol = (kBufs - 1) * kPAccStride + kTN;
+  static constexpr int kSfbCol = kSfaCol + 4 * kPKb;
+  static_assert(kSfbCol + 8 * kPKb <= kPTmemCols, "tensor memory layout");
+  // M = 256 (the pair), N = kTN, K = 64, E2M1 x E2M1, E8M0 scales, K-major
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kTN >> 3) << 17) | (1u << 23) |
+                                     ((uint32_t)(kPM >> 4) << 24);
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + kOutChunks * kPHalf * 128 + 256;
+  static_assert(kSmem <= 232448, "shared memory per CTA");
+};
 
 // Shared-memory descriptor of a K-major operand tile whose rows are 128 bytes
 // (K = 256 fp4), 128-byte swizzle: 8-row groups 1024 bytes apart.
@@ -494,16 +535,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-
-
-
-__host__ __device__ constexpr int pair_smem_bytes() {
-  return 1024 + kPStages * kPStageBytes + kPOutBytes + 256;
-}
-
-// M = 256 (the pair), N = 256, K = 64, E2M1 x E2M1, E8M0 scales, K-major.
-constexpr uint32_t kPIdescBase = (1u << 7) | (1u << 10) | ((uint32_t)(kPTile >> 3) << 17) | (1u << 23) |
-                                 ((uint32_t)(kPTile >> 4) << 24);
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -566,10 +597,14 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
       : "memory");
 }
 
+constexpr int kPEpiWarps = 8;                      // two per tensor-memory lane quarter
+constexpr int kPEpiThreads = 32 * kPEpiWarps;
+constexpr int kPThreads = 64 + kPEpiThreads;
+
 struct PairArgs {
   int M, N;
-  int k_steps;               // K / 128
-  int m_tiles, n_tiles;      // 256-row and 256-column tiles
+  int k_steps;               // stages of K per tile (K / 256)
+  int m_tiles, n_tiles;      // 256-row and kTN-column tiles
   int pairs;                 // clusters in the grid
 };
 
@@ -581,20 +616,22 @@ __device__ __forceinline__ void settle_ns(uint64_t ns) {
   while (global_timer_ns() - t0 < ns) {}
 }
 
-template <bool kBf16>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kBf16, int kTN>
+__global__ void __launch_bounds__(kPThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                  const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
                  const __grid_constant__ CUtensorMap ymap, const PairArgs args, unsigned int* devstat) {
+  using P = PairShape<kTN>;
+  constexpr int kS = P::kStages, kB = P::kBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* out_stage = smem + kPStages * kPStageBytes;           // 4 x [128 rows][128 B], 128B swizzle
-  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + kPOutBytes);
-  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kPStages]);
-  const uint32_t accf = smem_addr(&bars[2 * kPStages]), acce = smem_addr(&bars[2 * kPStages + 1]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kPStages + 2]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kPStages + 3]);
+  uint8_t* out_stage = smem + kS * P::kStageBytes;                // [128 rows][128 B] chunks, 128B swizzle
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + P::kOutChunks * kPHalf * 128);
+  const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[kS]);
+  const uint32_t accf0 = smem_addr(&bars[2 * kS]), acce0 = smem_addr(&bars[2 * kS + kB]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[2 * kS + 2 * kB]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[2 * kS + 2 * kB + 1]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();              // 0: issues the MMAs
@@ -611,12 +648,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
     tma_prefetch_desc(&sfamap);
     tma_prefetch_desc(&sfbmap);
     tma_prefetch_desc(&ymap);
-    for (int s = 0; s < kPStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(accf, 1);
-    mbar_init(acce, 2 * (kEpiThreads / 32));        // every epilogue warp of both CTAs
+    for (int b = 0; b < kB; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 2 * kPEpiWarps);           // every epilogue warp of both CTAs
+    }
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -641,24 +680,27 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
       for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
         const int t = pair + i * args.pairs;
         const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
-        const int arow = m_tile * kPTile + (int)rank * kPHalf;
-        const int brow = n_tile * kPTile + (int)rank * kPHalf;
-        const int sfa_blk = (m_tile * 2 + (int)rank) * KS128, sfb_blk = n_tile * 2 * KS128;
+        const int arow = m_tile * kPM + (int)rank * kPHalf;
+        const int bcol0 = n_tile * kTN;
+        const int brow = bcol0 + (int)rank * P::kBHalf;
+        // the 128-row scale blocks of A's rows of this CTA, and the first of
+        // the two that the tile's B rows meet
+        const int sfa_blk = (m_tile * 2 + (int)rank) * KS128, sfb_blk = (bcol0 >> 7) * KS128;
         for (int kt = 0; kt < KS; ++kt, ++seq) {
-          const int s = seq % kPStages;
-          if (seq >= kPStages && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(seq / kPStages - 1) & 1u)) {
+          const int s = seq % kS;
+          if (seq >= kS && !mbar_wait_bounded(empty0 + 8 * s, (uint32_t)(seq / kS - 1) & 1u)) {
             *abort_flag = 1;
             atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
             break;
           }
-          const uint32_t st = smem_addr(smem + s * kPStageBytes);
+          const uint32_t st = smem_addr(smem + s * P::kStageBytes);
           const uint32_t bar = map_to_rank(full0 + 8 * s, 0);
-          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)(2 * kPStageTx));
+          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)(2 * P::kStageTx));
           // codes, then the scale blocks of this stage's kPKb 128-K blocks: A's
-          // rows, then the first and the second 128 rows of B
+          // rows, then the two 128-row blocks of B
           tma_load_2d_pair(st, &amap, kt * (kPK / 2), arow, bar);
           tma_load_2d_pair(st + kPOpBytes, &bmap, kt * (kPK / 2), brow, bar);
-          const uint32_t sf = st + 2 * kPOpBytes;
+          const uint32_t sf = st + kPOpBytes + P::kBBytes;
           tma_load_2d_pair(sf, &sfamap, 0, sfa_blk + kPKb * kt, bar);
           tma_load_2d_pair(sf + kPKb * kSfBytes, &sfbmap, 0, sfb_blk + kPKb * kt, bar);
           tma_load_2d_pair(sf + 2 * kPKb * kSfBytes, &sfbmap, 0, sfb_blk + KS128 + kPKb * kt, bar);
@@ -670,32 +712,38 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
     if (lane == 0 && rank == 0) {
       int seq = 0;
       for (int i = 0; i < my_tiles; ++i) {
-        // both CTAs' epilogues have read the previous tile's accumulator
-        bool ok = i == 0 || mbar_wait_bounded(acce, (uint32_t)(i - 1) & 1u);
+        const int buf = i % kB, use = i / kB;
+        const int n_tile = (pair + i * args.pairs) / args.m_tiles;
+        // B scale of tile row 0 sits at row (n_tile kTN) % 128 of its block:
+        // 32 rows per tensor-memory column
+        const uint32_t sfb_shift = (uint32_t)(((n_tile * kTN) & 127) >> 5);
+        const uint32_t acc = tmem_base + (uint32_t)(buf * kPAccStride);
+        // both CTAs' epilogues have read this accumulator's previous tile
+        bool ok = use == 0 || mbar_wait_bounded(acce0 + 8 * buf, (uint32_t)(use - 1) & 1u);
         if (ok) fence_after_sync();
         for (int kt = 0; ok && kt < KS; ++kt, ++seq) {
-          const int s = seq % kPStages;
-          ok = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(seq / kPStages) & 1u) && !*abort_flag;
+          const int s = seq % kS;
+          ok = mbar_wait_bounded(full0 + 8 * s, (uint32_t)(seq / kS) & 1u) && !*abort_flag;
           if (!ok) break;
           fence_after_sync();
-          const uint32_t st = smem_addr(smem + s * kPStageBytes);
-          const uint32_t sf = st + 2 * kPOpBytes;
+          const uint32_t st = smem_addr(smem + s * P::kStageBytes);
+          const uint32_t sf = st + kPOpBytes + P::kBBytes;
 #pragma unroll
           for (int j = 0; j < kPKb; ++j) {
-            sf_copy_pair(tmem_base + kPSfaCol + 4 * j, sf_desc(sf + j * kSfBytes));
-            sf_copy_pair(tmem_base + kPSfbCol + 8 * j, sf_desc(sf + (kPKb + j) * kSfBytes));
-            sf_copy_pair(tmem_base + kPSfbCol + 8 * j + 4, sf_desc(sf + (2 * kPKb + j) * kSfBytes));
+            sf_copy_pair(tmem_base + P::kSfaCol + 4 * j, sf_desc(sf + j * kSfBytes));
+            sf_copy_pair(tmem_base + P::kSfbCol + 8 * j, sf_desc(sf + (kPKb + j) * kSfBytes));
+            sf_copy_pair(tmem_base + P::kSfbCol + 8 * j + 4, sf_desc(sf + (2 * kPKb + j) * kSfBytes));
           }
           // K = 64 per MMA: MMA kk reads scale block kk / 2, scales 2 (kk % 2) and 2 (kk % 2) + 1
 #pragma unroll
           for (int kk = 0; kk < 2 * kPKb; ++kk) {
             const int j = kk >> 1;
             const uint32_t sf_id = (uint32_t)(2 * (kk & 1));
-            const uint32_t sfa = (tmem_base + kPSfaCol + 4 * j) | (sf_id << 30);
-            const uint32_t sfb = (tmem_base + kPSfbCol + 8 * j) | (sf_id << 30);
-            const uint32_t idesc = kPIdescBase | (sf_id << 29) | (sf_id << 4);
-            mma_mxf4_pair(tmem_base, sw128_desc(st + kk * 32), sw128_desc(st + kPOpBytes + kk * 32),
-                          idesc, sfa, sfb, (kt | kk) != 0);
+            const uint32_t sfa = (tmem_base + P::kSfaCol + 4 * j) | (sf_id << 30);
+            const uint32_t sfb = (tmem_base + P::kSfbCol + 8 * j + sfb_shift) | (sf_id << 30);
+            const uint32_t idesc = P::kIdesc | (sf_id << 29) | (sf_id << 4);
+            mma_mxf4_pair(acc, sw128_desc(st + kk * 32), sw128_desc(st + kPOpBytes + kk * 32), idesc, sfa,
+                          sfb, (kt | kk) != 0);
           }
           mma_commit_pair(empty0 + 8 * s);
         }
@@ -704,90 +752,118 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
           atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
           break;
         }
-        mma_commit_pair(accf);
+        mma_commit_pair(accf0 + 8 * buf);
       }
       aborted = *abort_flag != 0;
     }
   } else {
-    // epilogue: warps 2..5 -> tensor-memory lane quarters (warp % 4); thread = one row
-    const int q = warp & 3;
+    // epilogue: warps 2 .. 2 + kPEpiWarps - 1.  Warp w reads tensor-memory
+    // lane quarter w % 4 (32 rows, one per thread) and half (w - 2) / 4 of
+    // the tile's columns in one round trip, hands the accumulator back, then
+    // stages Y in shared memory and writes it with TMA tensor stores.
+    constexpr int kHalfCols = kTN / 2;
+    constexpr int kCC = kBf16 ? 64 : 32;       // Y columns per staging chunk (128 bytes a row)
+    constexpr int kChunks = kTN / kCC;
+    constexpr int kW = kBf16 ? 8 : 4;          // Y columns per 16-byte group
+    const int q = warp & 3, h = (warp - 2) >> 2;
     const int etid = tid - 64;
     const int r_local = 32 * q + lane;
-    const uint32_t acce_leader = map_to_rank(acce, 0);
+    const int col0 = h * kHalfCols;
     for (int i = 0; i < my_tiles; ++i) {
+      const int buf = i % kB, use = i / kB;
       const int t = pair + i * args.pairs;
       const int m_tile = t % args.m_tiles, n_tile = t / args.m_tiles;
-      const int row0 = m_tile * kPTile + (int)rank * kPHalf, n0 = n_tile * kPTile;
-      const bool ok = mbar_wait_bounded(accf, (uint32_t)i & 1u);
+      const int row0 = m_tile * kPM + (int)rank * kPHalf, n0 = n_tile * kTN;
+      const bool ok = mbar_wait_bounded(accf0 + 8 * buf, (uint32_t)use & 1u);
       // the previous tile's stores have read the staging chunks
       if (etid == 0) bulk_wait_read_all();
-      if (epi_any(!ok || *abort_flag)) {
+      if (epi_any(!ok || *abort_flag, kPEpiThreads)) {
         if (!ok) atomicOr(devstat, (unsigned)KQ_DEVSTAT_WAIT_TIMEOUT);
         *abort_flag = 1;
         aborted = true;
         break;
       }
       fence_after_sync();
-      if constexpr (kBf16) {
-        // all 256 columns, as bf16, into the four chunks (64 columns = 128 B a row each)
-        for (int c = 0; c < kPTile / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
-          uint32_t w[16];
+      const uint32_t acc = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * kPAccStride + col0);
+      // 32-column loads (each starts at a multiple of 32 columns), one wait
+      uint32_t v[kHalfCols / 32][32];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const __nv_bfloat162 h2 =
-                __floats2bfloat162_rn(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
-            w[k] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-          if (c == kPTile / 32 - 1) {
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(acce_leader);
-          }
-          uint8_t* rowp = out_stage + (c >> 1) * (kPHalf * 128) + r_local * 128;
+      for (int g = 0; g < kHalfCols / 32; ++g) tmem_ld32_nowait(acc + 32 * g, v[g]);
+      tmem_wait_ld();
+      // keep every use of the loaded registers after the wait
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = (c & 1) * 4 + u;
-            *reinterpret_cast<uint4*>(rowp + ((j ^ (r_local & 7)) << 4)) =
-                make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      for (int g = 0; g < kHalfCols / 32; ++g)
+#pragma unroll
+        for (int k = 0; k < 32; ++k) asm volatile("" : "+r"(v[g][k]));
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(acce0 + 8 * buf, 0));
+      // Four 16-byte words of Y (columns a .. a + 4 kW / 4 - 1 of this warp's
+      // half) as they go to shared memory: fp32 bits, or bf16 pairs with the
+      // even column in the low half.
+      auto group = [&](int a, uint32_t (&w)[4]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (kBf16) {
+            const int b = a + 2 * e;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[b >> 5][b & 31]),
+                                                            __uint_as_float(v[(b + 1) >> 5][(b + 1) & 31]));
+            w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+          } else {
+            w[e] = v[(a + e) >> 5][(a + e) & 31];
           }
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        epi_barrier();
-        if (etid == 0) {
-          for (int h = 0; h < 4; ++h)
-            tma_store_2d(&ymap, n0 + 64 * h, row0, smem_addr(out_stage + h * (kPHalf * 128)));
-          bulk_commit();
-        }
-      } else {
-        // fp32: two halves of 128 columns (four chunks of 32 columns each)
-        for (int h = 0; h < 2; ++h) {
-          if (h == 1) {
+      };
+      if constexpr (kHalfCols % kCC == 0) {
+        // each half is whole chunks: per round, two chunks of each half
+        // (slots 2 h, 2 h + 1), so every register index is fixed at compile time
+        constexpr int kHC = kHalfCols / kCC;
+        static_assert(P::kOutChunks == 4, "two staging chunks per half and round");
+#pragma unroll
+        for (int a = 0; a < kHC; a += 2) {
+          if (a > 0) {
             if (etid == 0) bulk_wait_read_all();
-            epi_barrier();
+            epi_barrier(kPEpiThreads);
           }
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * h + 32 * c), r);
-            if (h == 1 && c == 3) {
-              fence_before_sync();
-              __syncwarp();
-              if (lane == 0) mbar_arrive_remote(acce_leader);
-            }
-            uint8_t* rowp = out_stage + c * (kPHalf * 128) + r_local * 128;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<uint4*>(rowp + ((u ^ (r_local & 7)) << 4)) =
-                  make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+          for (int cc = a; cc < a + 2 && cc < kHC; ++cc) {
+            uint8_t* rowp = out_stage + (2 * h + cc - a) * (kPHalf * 128) + r_local * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint32_t w[4];
+              group(cc * kCC + j * kW, w);
+              *reinterpret_cast<uint4*>(rowp + ((j ^ (r_local & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          epi_barrier();
+          epi_barrier(kPEpiThreads);
           if (etid == 0) {
-            for (int c = 0; c < 4; ++c)
-              tma_store_2d(&ymap, n0 + 128 * h + 32 * c, row0, smem_addr(out_stage + c * (kPHalf * 128)));
+            for (int hh = 0; hh < 2; ++hh)
+              for (int cc = a; cc < a + 2 && cc < kHC; ++cc)
+                tma_store_2d(&ymap, n0 + hh * kHalfCols + cc * kCC, row0,
+                             smem_addr(out_stage + (2 * hh + cc - a) * (kPHalf * 128)));
             bulk_commit();
           }
+        }
+      } else {
+        // halves split a chunk (bf16, 192 columns): chunks follow the tile,
+        // and both halves write into the shared one
+        static_assert(kChunks <= P::kOutChunks, "one round");
+#pragma unroll
+        for (int k = 0; k < kHalfCols / kW; ++k) {
+          const int c = col0 + k * kW;         // first Y column of this 16-byte group
+          uint32_t w[4];
+          group(k * kW, w);
+          const int j = (c % kCC) / kW;
+          uint8_t* rowp = out_stage + (c / kCC) * (kPHalf * 128) + r_local * 128;
+          *reinterpret_cast<uint4*>(rowp + ((j ^ (r_local & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        epi_barrier(kPEpiThreads);
+        if (etid == 0) {
+          for (int c = 0; c < kChunks; ++c)
+            tma_store_2d(&ymap, n0 + c * kCC, row0, smem_addr(out_stage + c * (kPHalf * 128)));
+          bulk_commit();
         }
       }
     }
@@ -874,14 +950,14 @@ int sf_tmap(CUtensorMap* tm, const uint8_t* tiled, int64_t rows, int64_t K) {
   return KQ_OK;
 }
 
-// Codes [rows][K/2] for the pair kernel: box 128 bytes (K = 256) x 128 rows,
-// 128-byte swizzle (the canonical K-major layout of 128-byte rows).
-int pair_codes_tmap(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t K) {
+// Codes [rows][K/2] for the pair kernel: box 128 bytes (K = 256) x box_rows
+// rows, 128-byte swizzle (the canonical K-major layout of 128-byte rows).
+int pair_codes_tmap(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = gemm_encoder();
   if (!enc) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled not found in the CUDA driver");
   const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
-  const cuuint32_t box[2] = {gemm::kPK / 2, gemm::kPHalf};
+  const cuuint32_t box[2] = {gemm::kPK / 2, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -890,41 +966,43 @@ int pair_codes_tmap(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t
   return KQ_OK;
 }
 
-// The CTA-pair kernel for M and N multiples of 256 and K a multiple of the
-// stage's K (no rank-1 term).
+// The CTA-pair kernel with kTN-column tiles, for M a multiple of 256, N of
+// kTN and K of the stage's K (no rank-1 term).
+template <int kTN>
 int gemm_pair_launch(const uint8_t* a_codes, const uint8_t* b_codes, const CUtensorMap& ym,
                      const uint8_t* a_sf_tiled, const uint8_t* b_sf_tiled, int64_t M, int64_t N,
                      int64_t K, bool bf16, unsigned int* devstat, cudaStream_t stream) {
+  using P = gemm::PairShape<kTN>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(KQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
-  const int smem = gemm::pair_smem_bytes();
+  const int smem = P::kSmem;
   static std::once_flag attr_once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
   std::call_once(attr_once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(gemm::gemm_pair_kernel<false>,
+    attr_err[dev] = cudaFuncSetAttribute(gemm::gemm_pair_kernel<false, kTN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (attr_err[dev] == cudaSuccess)
-      attr_err[dev] = cudaFuncSetAttribute(gemm::gemm_pair_kernel<true>,
+      attr_err[dev] = cudaFuncSetAttribute(gemm::gemm_pair_kernel<true, kTN>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute (pair)");
 
   CUtensorMap am, bm, sam, sbm;
-  if (int st = pair_codes_tmap(&am, a_codes, M, K)) return st;
-  if (int st = pair_codes_tmap(&bm, b_codes, N, K)) return st;
+  if (int st = pair_codes_tmap(&am, a_codes, M, K, gemm::kPHalf)) return st;
+  if (int st = pair_codes_tmap(&bm, b_codes, N, K, P::kBHalf)) return st;
   if (int st = sf_tmap(&sam, a_sf_tiled, M, K)) return st;
   if (int st = sf_tmap(&sbm, b_sf_tiled, N, K)) return st;
   gemm::PairArgs args;
   args.M = (int)M;
   args.N = (int)N;
   args.k_steps = (int)(K / gemm::kPK);
-  args.m_tiles = (int)(M / gemm::kPTile);
-  args.n_tiles = (int)(N / gemm::kPTile);
+  args.m_tiles = (int)(M / gemm::kPM);
+  args.n_tiles = (int)(N / kTN);
 
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(gemm::kThreads);
+  cfg.blockDim = dim3(gemm::kPThreads);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -936,7 +1014,7 @@ int gemm_pair_launch(const uint8_t* a_codes, const uint8_t* b_codes, const CUten
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  auto kern = bf16 ? gemm::gemm_pair_kernel<true> : gemm::gemm_pair_kernel<false>;
+  auto kern = bf16 ? gemm::gemm_pair_kernel<true, kTN> : gemm::gemm_pair_kernel<false, kTN>;
   // as many pairs as can be resident at once (one CTA per SM), no more than tiles
   int sms = 0;
   if (int st = sm_count(&sms)) return st;
@@ -1018,10 +1096,14 @@ int gemm_launch(const uint8_t* a_codes, const uint8_t* a_sf_tiled, const uint8_t
   }
   unsigned int* devstat = nullptr;
   if (int st = kq::device_status_address(&devstat)) return st;
-  if (M % kq::gemm::kPTile == 0 && N % kq::gemm::kPTile == 0 && K % kq::gemm::kPK == 0 &&
-      mu == nullptr && tma_store)
-    return kq::gemm_pair_launch(a_codes, b_codes, ym, a_sf_tiled, b_sf_tiled, M, N, K, bf16, devstat,
-                                kq::as_stream(stream));
+  if (M % kq::gemm::kPM == 0 && K % kq::gemm::kPK == 0 && mu == nullptr && tma_store) {
+    if (N % 256 == 0)
+      return kq::gemm_pair_launch<256>(a_codes, b_codes, ym, a_sf_tiled, b_sf_tiled, M, N, K, bf16, devstat,
+                                       kq::as_stream(stream));
+    if (N % 192 == 0)
+      return kq::gemm_pair_launch<192>(a_codes, b_codes, ym, a_sf_tiled, b_sf_tiled, M, N, K, bf16, devstat,
+                                       kq::as_stream(stream));
+  }
   kq::gemm::GemmArgs args;
   args.M = (int)M;
   args.N = (int)N;
