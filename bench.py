@@ -323,7 +323,8 @@ def ring_of(x0, n_slots: int, out_shapes):
 
 
 def time_per_config(kq, device, l2: int, names=("tiny", "pixart", "sana", "flux", "sweep")) -> dict:
-    """kq_quantize and sq_quantize on every BASELINE workload shape, and
+    """kq_quantize and sq_quantize on every workload shape (tiny, PixArt, SANA,
+    FLUX and the sweep), and
     kq_fold_weights on d x d weights for the sweep's widths: median
     per-launch device time of REPS bursts of LAUNCHES_PER_REP launches over
     an input ring larger than RING_FACTOR_L2 x L2."""
