@@ -476,14 +476,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
 // loads only into its own shared memory; the loads of both CTAs complete on
 // CTA 0's barrier, and CTA 0's MMA completions arrive on both CTAs' barriers.
 //
-// Tile width.  kTN = 192 (N a multiple of 192): two accumulators of 192
-// columns fit in tensor memory beside the scales, so the MMAs of the next tile
-// run while the epilogue drains the last one.  kTN = 256 (other N, multiples
-// of 256): one accumulator of 256 columns (two would leave no column for the
-// scales), handed back as soon as the epilogue has read it, before the
-// stores.  Scale blocks cover 128 B rows; a 192-column tile with an odd index
-// starts half-way through one, so it loads the two blocks it meets and points
-// the MMA's B-scale address two tensor-memory columns (64 rows) in.
+// Tile width.  kTN = 256 (N a multiple of 256): one accumulator of 256
+// columns (two would leave no column for the scales), handed back as soon as
+// the epilogue has read it, before the stores.  kTN = 192 (N a multiple of
+// 192 but not of 256): two accumulators of 192 columns fit beside the scales,
+// so the MMAs of the next tile run while the epilogue drains the last one;
+// where both widths apply the 256-wide tile wins, since the 192-wide one loads
+// 17 % more operand bytes per FLOP and the operand stream bounds the
+// mainloop.  Scale blocks cover 128 B rows; a 192-column tile with an odd
+// index starts half-way through one, so it loads the two blocks it meets and
+// points the MMA's B-scale address two tensor-memory columns (64 rows) in.
 //
 // A stage holds K = 256 (128-byte rows, 128-byte swizzle): per stage one
 // barrier round trip, six scale copies and four MMAs of K = 64.  With 64-byte
@@ -495,9 +497,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
 // owns tensor memory (both CTAs) and, in CTA 0, lane 0 issues the scale
 // copies and the MMAs; warps 2..9 read the accumulator (two warps per lane
 // quarter, one row per thread, half of the columns each, in one round trip),
-// hand it back, stage Y in shared memory and write it with TMA tensor stores.  Every wait is
-// bounded; a wait that runs out sets the device status word, the CTA drains,
-// meets its peer at the final cluster barrier and exits.
+// hand it back, stage Y in shared memory and write it with TMA tensor stores.
+// Every wait is bounded; a wait that runs out sets the device status word,
+// the CTA drains, meets its peer at the final cluster barrier and exits.
 constexpr int kPM = 256;                           // tile rows of a pair (the MMA's M)
 constexpr int kPHalf = 128;                        // rows of A in each CTA
 constexpr int kPK = 256;                           // K per stage (fp4 elements): 128-byte rows
