@@ -513,8 +513,10 @@ struct PairShape {
   static_assert(kTN == 192 || kTN == 256, "pair tile width");
   static constexpr int kBHalf = kTN / 2;                        // rows of B in each CTA
   static constexpr int kBufs = kTN == 256 ? 1 : 2;              // accumulators
-  static constexpr int kStages = kTN == 256 ? 4 : 5;
-  static constexpr int kOutChunks = 4;                          // [128 rows][128 B] staging chunks
+  static constexpr int kStages = 5;
+  // [128 rows][128 B] staging chunks: two for 256-wide tiles (Y leaves in
+  // rounds of two chunks; the stages take the rest of shared memory)
+  static constexpr int kOutChunks = kTN == 256 ? 2 : 4;
   static constexpr int kBBytes = kBHalf * kPK / 2;              // B codes per CTA per stage
   // bytes one CTA loads per stage: codes, A's scale blocks, two blocks of B scales
   static constexpr int kStageTx = kPOpBytes + kBBytes + 3 * kPKb * kSfBytes;
@@ -817,19 +819,20 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
         }
       };
       if constexpr (kHalfCols % kCC == 0) {
-        // each half is whole chunks: per round, two chunks of each half
-        // (slots 2 h, 2 h + 1), so every register index is fixed at compile time
+        // each half is whole chunks: per round, kPer chunks of each half
+        // (slots kPer h ..), so every register index is fixed at compile time
         constexpr int kHC = kHalfCols / kCC;
-        static_assert(P::kOutChunks == 4, "two staging chunks per half and round");
+        constexpr int kPer = P::kOutChunks / 2;
+        static_assert(P::kOutChunks % 2 == 0 && kPer >= 1, "whole staging chunks per half and round");
 #pragma unroll
-        for (int a = 0; a < kHC; a += 2) {
+        for (int a = 0; a < kHC; a += kPer) {
           if (a > 0) {
             if (etid == 0) bulk_wait_read_all();
             epi_barrier(kPEpiThreads);
           }
 #pragma unroll
-          for (int cc = a; cc < a + 2 && cc < kHC; ++cc) {
-            uint8_t* rowp = out_stage + (2 * h + cc - a) * (kPHalf * 128) + r_local * 128;
+          for (int cc = a; cc < a + kPer && cc < kHC; ++cc) {
+            uint8_t* rowp = out_stage + (kPer * h + cc - a) * (kPHalf * 128) + r_local * 128;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               uint32_t w[4];
@@ -841,9 +844,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
           epi_barrier(kPEpiThreads);
           if (etid == 0) {
             for (int hh = 0; hh < 2; ++hh)
-              for (int cc = a; cc < a + 2 && cc < kHC; ++cc)
+              for (int cc = a; cc < a + kPer && cc < kHC; ++cc)
                 tma_store_2d(&ymap, n0 + hh * kHalfCols + cc * kCC, row0,
-                             smem_addr(out_stage + (2 * hh + cc - a) * (kPHalf * 128)));
+                             smem_addr(out_stage + (kPer * hh + cc - a) * (kPHalf * 128)));
             bulk_commit();
           }
         }
